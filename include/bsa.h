@@ -1,0 +1,216 @@
+/*
+ * bsa.h — C ABI of libbsa: input-adaptive 3D block-sparse self-attention for
+ * video diffusion transformers on NVIDIA B200 (sm_100a).
+ *
+ * The operation is the head-wise sparse attention executor of
+ *   SPADE: An Input-Adaptive Sparse Attention Engine for Fast Video Diffusion
+ *   Models Inference (arXiv 2608.03335), §3.3 "Head-wise Sparse Attention":
+ *   Q, K, V are rearranged into a blocked layout by a 3D blocking scheme, one
+ *   mean summary (centroid) is formed per Q/K block, an inter-block importance
+ *   matrix is computed from the summaries and filtered by Top-K or Top-P, a
+ *   flash block-sparse attention kernel computes softmax(QK^T/sqrt(d) + M)V
+ *   (§2.2, Eq. (2)) over the selected block pairs, and the output blocks are
+ *   restored to the original token order.
+ * Block shapes follow the DecoupAttn Plans README ("Contents" table: block
+ * shape = frames x rows x cols of one key block). Density follows the blog
+ * "Does sparse attention actually speed up video generation?" ("How this was
+ * measured": the fraction of key blocks each query block keeps).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every tensor pointer is DEVICE memory owned by the caller, contiguous,
+ *    16-byte aligned, on the current CUDA device.  `stream` is a cudaStream_t
+ *    (NULL = legacy default stream).  Calls are asynchronous on that stream:
+ *    host-side validation happens first, and a call that returns anything but
+ *    BSA_OK has launched nothing and written nothing.
+ *  - Element type of Q/K/V/O and of the blocked tensors is the plan's dtype
+ *    (BSA_F32: float, BSA_BF16: __nv_bfloat16).  Centroids and scores are
+ *    float.  Index lists are int32.
+ *  - Token layout ("original order") of Q/K/V/O: [B, Ntot, Hd, D] with
+ *    Ntot = T*H*W + n_text.  Video token (t, y, x) sits at n = (t*H + y)*W + x
+ *    (frame-major raster, the DiT flattening of SPADE §2.1); text token u sits
+ *    at n = T*H*W + u.
+ *  - Blocked layout: [B, Hd, Npad_tot, D], Npad_tot = (nb + nb_text) * bs.
+ *    The grid is padded at the high end of each axis to Tp = ceil(T/bf)*bf
+ *    (likewise Hp, Wp).  Video block (tb, yb, xb) has id
+ *    (tb*nby + yb)*nbx + xb; inside a block, slot (dt, dy, dx) is
+ *    (dt*br + dy)*bc + dx.  Text tokens fill nb_text = ceil(n_text/bs)
+ *    trailing blocks (ids nb .. nb+nb_text-1) in order.  Pad slots hold 0,
+ *    are never attended as keys, and produce output 0 as queries.
+ *  - Text key blocks are attended by every query; text query blocks attend
+ *    every key block (dense rows).  Text blocks take no part in scoring.
+ *  - Errors: every call returns a bsa_status; bsa_last_error_string() gives a
+ *    thread-local message for the last failure.
+ */
+#ifndef BSA_H_
+#define BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BSA_VERSION 100
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1, /* bad shape, pointer, parameter or list width   */
+  BSA_ERR_UNSUPPORTED = 2, /* valid request this build cannot serve          */
+  BSA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed              */
+  BSA_ERR_TIMEOUT = 4,     /* a bounded in-kernel wait ran out (dev_status)  */
+  BSA_ERR_WORKSPACE = 5,   /* workspace missing or smaller than required     */
+  BSA_ERR_BAD_INDEX = 6    /* an index list entry was out of range (skipped) */
+} bsa_status;
+
+typedef enum { BSA_F32 = 0, BSA_BF16 = 1 } bsa_dtype;
+
+/* Selection rule of the inter-block estimator (SPADE §3.1 "Top-K/Top-P
+ * mode", §3.3 "Scores are filtered by Top-K or Top-P").
+ *  BSA_TOPK: per head h, keep k_h = ceil(rho_h * nb - 1e-9) (clamped to
+ *            [1, nb]) video key blocks with the largest centroid scores;
+ *            param = rho_h, the density in (0, 1].
+ *  BSA_TOPP: per head h, keep the shortest prefix, in descending score
+ *            order, whose softmax mass reaches tau_h; param = tau_h in (0, 1].
+ * Equal scores are ordered by ascending key-block index. */
+typedef enum { BSA_TOPK = 0, BSA_TOPP = 1 } bsa_select_mode;
+
+typedef struct bsa_plan_s* bsa_plan_t;
+
+/* Derived sizes of a plan (all counts per batch element and head). */
+typedef struct {
+  int batch, T, H, W, bf, br, bc, heads, head_dim, n_text;
+  int dtype;            /* bsa_dtype                                        */
+  int Tp, Hp, Wp;       /* padded grid                                      */
+  int nbt, nby, nbx;    /* blocks per axis                                  */
+  int nb;               /* video blocks = nbt*nby*nbx                       */
+  int nb_text;          /* text blocks = ceil(n_text / bs)                  */
+  int bs;               /* tokens per block = bf*br*bc                      */
+  long long n_video;    /* T*H*W                                            */
+  long long n_tot;      /* n_video + n_text (rows of the original layout)   */
+  long long npad_tot;   /* (nb + nb_text) * bs (rows of the blocked layout) */
+  int attn_path;        /* 1 = tcgen05 tensor-core path, 0 = fp32 SIMT path */
+} bsa_plan_info_t;
+
+/* bsa_plan_create — describe one attention problem (SPADE §3 "Let the head
+ * dimension be d_head ... BS the block size and NB the number of blocks";
+ * §3.1 blocking schemes, Fig. 3).
+ *   batch >= 1; T, H, W >= 1 (latent frames, rows, cols); bf, br, bc >= 1
+ *   (block extent per axis, at most the padded grid); heads >= 1;
+ *   head_dim in {64, 128}; n_text >= 0 trailing text tokens; dtype.
+ *   Block size bs = bf*br*bc must be in [1, 256].  The tensor-core path
+ *   serves dtype BSA_BF16 with bs == 128; every other valid plan runs the
+ *   fp32 SIMT path (exact fp32 arithmetic, slower).
+ * Ownership: the plan is library-owned and immutable; it holds a few bytes of
+ * device memory on the device current at creation (status word).  Destroy it
+ * with bsa_plan_destroy on the same device. */
+bsa_status bsa_plan_create(bsa_plan_t* out, int batch, int T, int H, int W,
+                           int bf, int br, int bc, int heads, int head_dim,
+                           int n_text, bsa_dtype dtype);
+bsa_status bsa_plan_destroy(bsa_plan_t plan);
+bsa_status bsa_plan_get_info(bsa_plan_t plan, bsa_plan_info_t* info);
+
+/* bsa_kmax_for — the index-list width that every selection under `mode` and
+ * the host array param_per_head[heads] fits in: max_h k_h + nb_text for
+ * BSA_TOPK, nb + nb_text for BSA_TOPP.  Validates the parameters. */
+bsa_status bsa_kmax_for(bsa_plan_t plan, bsa_select_mode mode,
+                        const double* param_per_head, int* kmax);
+
+/* bsa_workspace_size — bytes of device workspace that bsa_select and
+ * bsa_forward need for list width kmax. */
+bsa_status bsa_workspace_size(bsa_plan_t plan, int kmax, size_t* select_ws,
+                              size_t* forward_ws);
+
+/* bsa_permute — layout transform into the blocked layout (SPADE §3.3,
+ * "rearranged into a blocked layout by the Selected Blocking Scheme"),
+ * optionally fused with the mean summarizer (§3.3 "Operator fusion";
+ * MEAN-SPADE, §3.1 (q_mean, k_mean)).
+ *   x         [B, Ntot, Hd, D]      input in original order (read only)
+ *   x_blk     [B, Hd, Npad_tot, D]  output, pad slots written as 0
+ *   centroids [B, Hd, nb, D] float  optional (NULL = skip): per video block,
+ *             the mean over its valid tokens, summed in fp32.
+ * bsa_permute_qkv does Q, K and V in one launch (centroids for Q and K). */
+bsa_status bsa_permute(bsa_plan_t plan, const void* x, void* x_blk,
+                       float* centroids, void* stream);
+bsa_status bsa_permute_qkv(bsa_plan_t plan, const void* q, const void* k,
+                           const void* v, void* q_blk, void* k_blk,
+                           void* v_blk, float* q_cent, float* k_cent,
+                           void* stream);
+
+/* bsa_unpermute — restore blocked output to the original token order (SPADE
+ * §3.3, "output blocks are restored to the original layout"); pad slots are
+ * dropped.   o_blk [B, Hd, Npad_tot, D] -> o [B, Ntot, Hd, D]. */
+bsa_status bsa_unpermute(bsa_plan_t plan, const void* o_blk, void* o,
+                         void* stream);
+
+/* bsa_select — index search (SPADE §3.3: summaries Q', K' of shape
+ * (N_blocks, d_head); inter-block importance N_Qb x N_Kb; Top-K / Top-P).
+ *   q_blk, k_blk  blocked Q and K (plan dtype)
+ *   mode, param_per_head  host array [Hd] of densities or thresholds
+ *   kmax          list width (>= bsa_kmax_for result)
+ *   idx  [B, Hd, nb, kmax] int32 out: per video query block, the selected
+ *        video key blocks in ascending id, then the nb_text text key blocks;
+ *        entries past cnt are left untouched
+ *   cnt  [B, Hd, nb] int32 out: list length (selected video blocks + nb_text)
+ *   scores [B, Hd, nb, nb] float out, optional (NULL = skip): the row-softmax
+ *        p_ij = softmax_j(qbar_i . kbar_j / sqrt(D)) computed in fp32
+ *   ws, ws_bytes  device workspace of at least select_ws bytes (centroids)
+ * Text query blocks have no list: they attend densely. */
+bsa_status bsa_select(bsa_plan_t plan, const void* q_blk, const void* k_blk,
+                      bsa_select_mode mode, const double* param_per_head,
+                      int kmax, int32_t* idx, int32_t* cnt, float* scores,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* bsa_select_centroids — bsa_select from precomputed fp32 centroids
+ * [B, Hd, nb, D] (as written by bsa_permute); needs no workspace. */
+bsa_status bsa_select_centroids(bsa_plan_t plan, const float* q_cent,
+                                const float* k_cent, bsa_select_mode mode,
+                                const double* param_per_head, int kmax,
+                                int32_t* idx, int32_t* cnt, float* scores,
+                                void* stream);
+
+/* bsa_attention — flash block-sparse attention (SPADE §2.2 Eq. (2) with M = 0
+ * on selected block pairs and valid keys, -inf elsewhere; §3.3 (3): online
+ * softmax, no dense score matrix).
+ *   q_blk, k_blk, v_blk  blocked inputs;  o_blk  blocked output (pad rows 0)
+ *   idx, cnt, kmax       lists as written by bsa_select (any ascending list
+ *                        of distinct ids in [0, nb+nb_text) is accepted)
+ *   dev_status           optional int32 device word (NULL = plan-owned):
+ *                        0 on success, BSA_ERR_TIMEOUT if a bounded wait ran
+ *                        out, BSA_ERR_BAD_INDEX if a list entry was out of
+ *                        range (that entry is skipped).  The caller reads it
+ *                        after synchronising; bsa_check_status does that for
+ *                        the plan-owned word.
+ * Output rows are softmax-weighted sums accumulated in fp32 and rounded to
+ * the plan dtype (round to nearest even). */
+bsa_status bsa_attention(bsa_plan_t plan, const void* q_blk, const void* k_blk,
+                         const void* v_blk, const int32_t* idx,
+                         const int32_t* cnt, int kmax, void* o_blk,
+                         int32_t* dev_status, void* stream);
+
+/* bsa_forward — the whole executor on one stream: permute (+centroids) ->
+ * select -> attention -> unpermute (SPADE §3.3, Fig. 2(c)).
+ *   q, k, v, o        original-order tensors [B, Ntot, Hd, D]
+ *   idx_out, cnt_out  optional copies of the lists (NULL = keep internal)
+ *   kmax              list width (>= bsa_kmax_for result)
+ *   ws, ws_bytes      device workspace of at least forward_ws bytes */
+bsa_status bsa_forward(bsa_plan_t plan, const void* q, const void* k,
+                       const void* v, bsa_select_mode mode,
+                       const double* param_per_head, int kmax, void* o,
+                       int32_t* idx_out, int32_t* cnt_out, void* ws,
+                       size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* bsa_check_status — synchronise `stream`, read and clear the plan-owned
+ * status word; returns BSA_OK or the recorded error. */
+bsa_status bsa_check_status(bsa_plan_t plan, void* stream);
+
+/* Thread-local message describing the last non-OK return of this thread. */
+const char* bsa_last_error_string(void);
+int bsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H_ */

@@ -1,0 +1,370 @@
+// oracle.cpp — plain, slow, fp64 CPU oracle of 3D block-sparse attention.
+//
+// TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
+// cpu_baseline / reference legs of bench.py may load or call this code.  The
+// product path (libbsa and its Python binding) never touches it, and this file
+// shares no code, header, table or constant with the CUDA implementation.
+//
+// What it computes is the head-wise sparse attention executor of
+//   SPADE: An Input-Adaptive Sparse Attention Engine for Fast Video Diffusion
+//   Models Inference, §3.3 "Head-wise Sparse Attention":
+//     blocked layout -> one mean summary per Q/K block -> inter-block
+//     importance matrix -> Top-K / Top-P -> block-sparse attention (§2.2,
+//     Eq. (2)) -> output restored to the original layout,
+// with the block-shape convention of the DecoupAttn Plans README ("Contents":
+// frames x rows x cols of one key block) and the density of the blog "Does
+// sparse attention actually speed up video generation?" ("How this was
+// measured": the fraction of key blocks each query block keeps).
+//
+// Every quantity is computed by its plain definition in double precision,
+// one element at a time, with no blocking, fusion or reordering.  Inputs are
+// float arrays (bf16 inputs are widened to float exactly by the caller).
+//
+// Readings of points the pages leave open (each one is listed in the design
+// notes of the repository):
+//   R1 token order: video token (t,y,x) at n = (t*H + y)*W + x (SPADE §2.1,
+//      the latent is flattened to a 1D sequence); text tokens follow.
+//   R2 block order (tb,yb,xb) raster; slot order (dt,dy,dx) raster; the grid
+//      is padded at the high end of each axis; pad slots are 0, are never
+//      keys and give output 0 as queries.
+//   R3 centroid = arithmetic mean over the valid tokens of a block.
+//   R4 inter-block score s_ij = qbar_i . kbar_j / sqrt(D), p_i = softmax_j(s_i)
+//      over the nb video key blocks.
+//   R5 k = ceil(rho * nb - 1e-9) clamped to [1, nb].
+//   R6 order for selection: p descending, then key-block id ascending.
+//   R7 Top-P: the smallest m >= 1 whose descending prefix mass reaches tau.
+//   R8 text blocks are not scored; every video query block also attends all
+//      text key blocks; text query tokens attend every token.
+//   R9 lists are stored in ascending block id, text blocks last.
+//
+// Geometry array g[10] = {B, T, H, W, bf, br, bc, Hd, D, n_text}.
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+namespace {
+
+struct Geom {
+  long long B, T, H, W, bf, br, bc, Hd, D, n_text;
+  long long nbt, nby, nbx, nb, bs, nb_text, n_video, n_tot, npad_tot;
+};
+
+Geom make_geom(const int* g) {
+  Geom G;
+  G.B = g[0]; G.T = g[1]; G.H = g[2]; G.W = g[3];
+  G.bf = g[4]; G.br = g[5]; G.bc = g[6]; G.Hd = g[7]; G.D = g[8];
+  G.n_text = g[9];
+  G.nbt = (G.T + G.bf - 1) / G.bf;
+  G.nby = (G.H + G.br - 1) / G.br;
+  G.nbx = (G.W + G.bc - 1) / G.bc;
+  G.nb = G.nbt * G.nby * G.nbx;
+  G.bs = G.bf * G.br * G.bc;
+  G.nb_text = (G.n_text + G.bs - 1) / G.bs;
+  G.n_video = G.T * G.H * G.W;
+  G.n_tot = G.n_video + G.n_text;
+  G.npad_tot = (G.nb + G.nb_text) * G.bs;
+  return G;
+}
+
+int n_threads() {
+  const char* e = std::getenv("ORACLE_THREADS");
+  if (e && std::atoi(e) > 0) return std::atoi(e);
+  unsigned h = std::thread::hardware_concurrency();
+  return h ? (int)h : 1;
+}
+
+// Runs f(i) for i in [0, n) on all threads, static interleaved split.
+template <class F>
+void parallel_for(long long n, F f) {
+  int nt = n_threads();
+  if (nt > n) nt = (int)std::max<long long>(n, 1);
+  std::vector<std::thread> pool;
+  for (int t = 0; t < nt; ++t)
+    pool.emplace_back([=, &f] {
+      for (long long i = t; i < n; i += nt) f(i);
+    });
+  for (auto& th : pool) th.join();
+}
+
+// Block id and slot of a video token (t, y, x): read R2 in the token -> slot
+// direction.
+void video_slot(const Geom& G, long long t, long long y, long long x,
+                long long* blk, long long* slot) {
+  long long tb = t / G.bf, dt = t % G.bf;
+  long long yb = y / G.br, dy = y % G.br;
+  long long xb = x / G.bc, dx = x % G.bc;
+  *blk = (tb * G.nby + yb) * G.nbx + xb;
+  *slot = (dt * G.br + dy) * G.bc + dx;
+}
+
+// Original token index of every valid token of block j (video or text).
+std::vector<long long> block_tokens(const Geom& G, long long j) {
+  std::vector<long long> out;
+  if (j < G.nb) {
+    long long tb = j / (G.nby * G.nbx);
+    long long yb = (j / G.nbx) % G.nby;
+    long long xb = j % G.nbx;
+    for (long long dt = 0; dt < G.bf; ++dt)
+      for (long long dy = 0; dy < G.br; ++dy)
+        for (long long dx = 0; dx < G.bc; ++dx) {
+          long long t = tb * G.bf + dt, y = yb * G.br + dy, x = xb * G.bc + dx;
+          if (t < G.T && y < G.H && x < G.W) out.push_back((t * G.H + y) * G.W + x);
+        }
+  } else {
+    long long u0 = (j - G.nb) * G.bs;
+    for (long long u = u0; u < u0 + G.bs && u < G.n_text; ++u)
+      out.push_back(G.n_video + u);
+  }
+  return out;
+}
+
+}  // namespace
+
+extern "C" {
+
+int orc_threads(void) { return n_threads(); }
+
+// Layout transform (SPADE §3.3: Q, K, V "rearranged into a blocked layout").
+// x [B, Ntot, Hd, D] -> x_blk [B, Hd, Npad_tot, D]; pad slots are 0 (R2).
+void orc_permute(const int* g, const float* x, double* x_blk) {
+  Geom G = make_geom(g);
+  std::memset(x_blk, 0, sizeof(double) * G.B * G.Hd * G.npad_tot * G.D);
+  for (long long b = 0; b < G.B; ++b)
+    for (long long n = 0; n < G.n_tot; ++n) {
+      long long blk, slot;
+      if (n < G.n_video) {
+        long long t = n / (G.H * G.W), y = (n / G.W) % G.H, xx = n % G.W;
+        video_slot(G, t, y, xx, &blk, &slot);
+      } else {
+        blk = G.nb + (n - G.n_video) / G.bs;
+        slot = (n - G.n_video) % G.bs;
+      }
+      for (long long h = 0; h < G.Hd; ++h)
+        for (long long d = 0; d < G.D; ++d)
+          x_blk[((b * G.Hd + h) * G.npad_tot + blk * G.bs + slot) * G.D + d] =
+              (double)x[((b * G.n_tot + n) * G.Hd + h) * G.D + d];
+    }
+}
+
+// Inverse layout transform (SPADE §3.3: "output blocks are restored to the
+// original layout"); pad slots are dropped.
+void orc_unpermute(const int* g, const double* x_blk, double* x) {
+  Geom G = make_geom(g);
+  for (long long b = 0; b < G.B; ++b)
+    for (long long n = 0; n < G.n_tot; ++n) {
+      long long blk, slot;
+      if (n < G.n_video) {
+        long long t = n / (G.H * G.W), y = (n / G.W) % G.H, xx = n % G.W;
+        video_slot(G, t, y, xx, &blk, &slot);
+      } else {
+        blk = G.nb + (n - G.n_video) / G.bs;
+        slot = (n - G.n_video) % G.bs;
+      }
+      for (long long h = 0; h < G.Hd; ++h)
+        for (long long d = 0; d < G.D; ++d)
+          x[((b * G.n_tot + n) * G.Hd + h) * G.D + d] =
+              x_blk[((b * G.Hd + h) * G.npad_tot + blk * G.bs + slot) * G.D + d];
+    }
+}
+
+// Mean summarizer (SPADE §3.1 MEAN-SPADE, (q_mean, k_mean); §3.3 summaries
+// Q', K' of shape (N_blocks, d_head)); R3: mean over valid tokens.
+// x [B, Ntot, Hd, D] -> cent [B, Hd, nb, D].
+void orc_centroids(const int* g, const float* x, double* cent) {
+  Geom G = make_geom(g);
+  std::vector<long long> count(G.nb, 0);
+  std::memset(cent, 0, sizeof(double) * G.B * G.Hd * G.nb * G.D);
+  for (long long n = 0; n < G.n_video; ++n) {
+    long long t = n / (G.H * G.W), y = (n / G.W) % G.H, xx = n % G.W, blk, slot;
+    video_slot(G, t, y, xx, &blk, &slot);
+    count[blk] += 1;
+    for (long long b = 0; b < G.B; ++b)
+      for (long long h = 0; h < G.Hd; ++h)
+        for (long long d = 0; d < G.D; ++d)
+          cent[((b * G.Hd + h) * G.nb + blk) * G.D + d] +=
+              (double)x[((b * G.n_tot + n) * G.Hd + h) * G.D + d];
+  }
+  for (long long b = 0; b < G.B; ++b)
+    for (long long h = 0; h < G.Hd; ++h)
+      for (long long blk = 0; blk < G.nb; ++blk)
+        for (long long d = 0; d < G.D; ++d)
+          cent[((b * G.Hd + h) * G.nb + blk) * G.D + d] /= (double)count[blk];
+}
+
+// Inter-block estimator (SPADE §3.1 "the dot product of blue vectors gives
+// inter-block importance", §3.3 N_Qb x N_Kb matrix); R4:
+// p[b,h,i,j] = softmax_j( qbar_i . kbar_j / sqrt(D) ).
+void orc_scores(const int* g, const double* qc, const double* kc, double* p) {
+  Geom G = make_geom(g);
+  const double scale = 1.0 / std::sqrt((double)G.D);
+  parallel_for(G.B * G.Hd * G.nb, [&](long long row) {
+    long long bh = row / G.nb;
+    const double* q = qc + row * G.D;
+    double* out = p + row * G.nb;
+    double m = -INFINITY;
+    for (long long j = 0; j < G.nb; ++j) {
+      const double* k = kc + (bh * G.nb + j) * G.D;
+      double s = 0.0;
+      for (long long d = 0; d < G.D; ++d) s += q[d] * k[d];
+      out[j] = s * scale;
+      m = std::max(m, out[j]);
+    }
+    double z = 0.0;
+    for (long long j = 0; j < G.nb; ++j) {
+      out[j] = std::exp(out[j] - m);
+      z += out[j];
+    }
+    for (long long j = 0; j < G.nb; ++j) out[j] /= z;
+  });
+}
+
+// Number of key blocks a density keeps (R5; the blog's "fraction of key
+// blocks each query block keeps").
+int orc_k_for_density(double rho, int nb) {
+  long long k = (long long)std::ceil(rho * (double)nb - 1e-9);
+  if (k < 1) k = 1;
+  if (k > nb) k = nb;
+  return (int)k;
+}
+
+// Top-K / Top-P selection (SPADE §3.1 "Top-K/Top-P mode"; §3.3 "Scores are
+// filtered by Top-K or Top-P"; inter-top value = "Top-P cumulative threshold
+// or Top-K keep").  mode 0 = top-k with params[h] = density, mode 1 = top-p
+// with params[h] = tau.  Lists: ascending video ids then text ids (R8, R9).
+// tie[row] = 1 where the decision is within the 1e-5 relative tolerance of
+// flipping (R6/R7 boundary), else 0.
+void orc_select(const int* g, const double* p, int mode, const double* params,
+                int kmax, int* idx, int* cnt, int* tie) {
+  Geom G = make_geom(g);
+  parallel_for(G.B * G.Hd * G.nb, [&](long long row) {
+    long long h = (row / G.nb) % G.Hd;
+    const double* pr = p + row * G.nb;
+    std::vector<long long> order(G.nb);
+    for (long long j = 0; j < G.nb; ++j) order[j] = j;
+    std::sort(order.begin(), order.end(), [&](long long a, long long b) {
+      if (pr[a] != pr[b]) return pr[a] > pr[b];
+      return a < b;
+    });
+    long long m;
+    int is_tie = 0;
+    if (mode == 0) {
+      m = orc_k_for_density(params[h], (int)G.nb);
+      if (m < G.nb) {
+        double a = pr[order[m - 1]], b = pr[order[m]];
+        if (std::fabs(a - b) <= 1e-5 * std::fabs(a)) is_tie = 1;
+      }
+    } else {
+      double tau = params[h], cum = 0.0, before = 0.0;
+      m = 0;
+      while (m < G.nb) {
+        before = cum;
+        cum += pr[order[m]];
+        ++m;
+        if (cum >= tau) break;
+      }
+      if (std::fabs(before - tau) <= 1e-5 * tau) is_tie = 1;
+      if (std::fabs(cum - tau) <= 1e-5 * tau) is_tie = 1;
+      if (m < G.nb) {
+        double a = pr[order[m - 1]], b = pr[order[m]];
+        if (std::fabs(a - b) <= 1e-5 * std::fabs(a)) is_tie = 1;
+      }
+    }
+    std::vector<long long> chosen(order.begin(), order.begin() + m);
+    std::sort(chosen.begin(), chosen.end());
+    int* out = idx + row * kmax;
+    long long c = 0;
+    for (long long j : chosen) out[c++] = (int)j;
+    for (long long t = 0; t < G.nb_text; ++t) out[c++] = (int)(G.nb + t);
+    cnt[row] = (int)c;
+    tie[row] = is_tie;
+  });
+}
+
+// Block-sparse attention (SPADE §2.2, Eq. (2)): for each valid query token,
+// softmax(q.k/sqrt(D)) over the union of the valid keys of its selected key
+// blocks (M = 0 there, -inf elsewhere), applied to V; §2.2 Eq. (1) for text
+// query tokens, which attend every token (R8).  Works on the ORIGINAL layout.
+//   rows: NULL = every token (o is [B, Ntot, Hd, D]); otherwise n_rows token
+//   indices, and o is [B, n_rows, Hd, D].
+void orc_attention(const int* g, const float* q, const float* k, const float* v,
+                   const int* idx, const int* cnt, int kmax,
+                   const long long* rows, long long n_rows, double* o) {
+  Geom G = make_geom(g);
+  const double scale = 1.0 / std::sqrt((double)G.D);
+  long long nr = rows ? n_rows : G.n_tot;
+  parallel_for(G.B * G.Hd * nr, [&](long long task) {
+    long long b = task / (G.Hd * nr);
+    long long h = (task / nr) % G.Hd;
+    long long r = task % nr;
+    long long n = rows ? rows[r] : r;
+    // The set of key tokens this query may attend.
+    std::vector<long long> keys;
+    if (n < G.n_video) {
+      long long t = n / (G.H * G.W), y = (n / G.W) % G.H, xx = n % G.W, blk, slot;
+      video_slot(G, t, y, xx, &blk, &slot);
+      const int* list = idx + ((b * G.Hd + h) * G.nb + blk) * kmax;
+      int c = cnt[(b * G.Hd + h) * G.nb + blk];
+      for (int e = 0; e < c; ++e) {
+        std::vector<long long> tk = block_tokens(G, list[e]);
+        keys.insert(keys.end(), tk.begin(), tk.end());
+      }
+    } else {
+      for (long long j = 0; j < G.nb + G.nb_text; ++j) {
+        std::vector<long long> tk = block_tokens(G, j);
+        keys.insert(keys.end(), tk.begin(), tk.end());
+      }
+    }
+    const float* qv = q + ((b * G.n_tot + n) * G.Hd + h) * G.D;
+    std::vector<double> s(keys.size());
+    double m = -INFINITY;
+    for (size_t c = 0; c < keys.size(); ++c) {
+      const float* kv = k + ((b * G.n_tot + keys[c]) * G.Hd + h) * G.D;
+      double acc = 0.0;
+      for (long long d = 0; d < G.D; ++d) acc += (double)qv[d] * (double)kv[d];
+      s[c] = acc * scale;
+      m = std::max(m, s[c]);
+    }
+    double z = 0.0;
+    for (size_t c = 0; c < keys.size(); ++c) {
+      s[c] = std::exp(s[c] - m);
+      z += s[c];
+    }
+    double* out = o + ((b * nr + r) * G.Hd + h) * G.D;
+    for (long long d = 0; d < G.D; ++d) out[d] = 0.0;
+    for (size_t c = 0; c < keys.size(); ++c) {
+      const float* vv = v + ((b * G.n_tot + keys[c]) * G.Hd + h) * G.D;
+      double w = s[c] / z;
+      for (long long d = 0; d < G.D; ++d) out[d] += w * (double)vv[d];
+    }
+  });
+}
+
+// Number of (query token, key token) pairs the lists select, valid tokens
+// only, per batch element and head summed (SPADE §4.1 "Sparsity — fraction of
+// pruned attention scores"; effective FLOPs = 4 * pairs * D).
+long long orc_selected_pairs(const int* g, const int* idx, const int* cnt,
+                             int kmax) {
+  Geom G = make_geom(g);
+  std::vector<long long> valid(G.nb + G.nb_text);
+  for (long long j = 0; j < G.nb + G.nb_text; ++j)
+    valid[j] = (long long)block_tokens(G, j).size();
+  long long total = 0;
+  for (long long bh = 0; bh < G.B * G.Hd; ++bh) {
+    for (long long i = 0; i < G.nb; ++i) {
+      long long keys = 0;
+      const int* list = idx + (bh * G.nb + i) * kmax;
+      for (int e = 0; e < cnt[bh * G.nb + i]; ++e) keys += valid[list[e]];
+      total += keys * valid[i];
+    }
+    for (long long i = G.nb; i < G.nb + G.nb_text; ++i)
+      total += valid[i] * G.n_tot;
+  }
+  return total;
+}
+
+}  // extern "C"

@@ -1,0 +1,286 @@
+"""Pins of the fp64 oracle against things other than itself (CPU only).
+
+Each test ties one oracle function to an independent statement of what the
+pages fix: a numpy reshape/transpose formulation of the blocked layout
+(SPADE §3.3 layout transform; DecoupAttn Plans README block shapes
+"frames x rows x cols"), brute-force means (SPADE §3.1 MEAN-SPADE), scipy's
+softmax (SPADE §3.3 inter-block matrix), exhaustive subset search for Top-K
+and Top-P (SPADE §3.1 "Top-K/Top-P mode"), torch's fp64 scaled-dot-product
+attention, dense (SPADE §2.2 Eq. (1)) and with an explicit token mask
+(Eq. (2)), and closed forms (V = 1 gives O = 1; equal keys give the plain
+mean of the allowed values).
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- helpers --
+def token_table(g):
+    """[nb + nb_text, bs] original token id of every slot, -1 for pad.
+
+    Built by padding a (T,H,W) id grid and splitting it with reshape/transpose:
+    block (tb,yb,xb) raster, slot (dt,dy,dx) raster; text blocks follow.
+    """
+    Tp, Hp, Wp = g.nbt * g.bf, g.nby * g.br, g.nbx * g.bc
+    ids = np.full((Tp, Hp, Wp), -1, dtype=np.int64)
+    ids[:g.T, :g.H, :g.W] = np.arange(g.n_video).reshape(g.T, g.H, g.W)
+    blocks = ids.reshape(g.nbt, g.bf, g.nby, g.br, g.nbx, g.bc).transpose(0, 2, 4, 1, 3, 5)
+    blocks = blocks.reshape(g.nb, g.bs)
+    text = np.full(g.nb_text * g.bs, -1, dtype=np.int64)
+    text[:g.n_text] = g.n_video + np.arange(g.n_text)
+    return np.concatenate([blocks, text.reshape(g.nb_text, g.bs)], axis=0)
+
+
+def rand_x(g, seed):
+    return np.random.default_rng(seed).standard_normal((g.B, g.n_tot, g.Hd, g.D)).astype(np.float32)
+
+
+def token_mask(g, idx, cnt):
+    """[B, Hd, Ntot, Ntot] boolean: query token may attend key token."""
+    tab = token_table(g)
+    blk_of = np.empty(g.n_tot, dtype=np.int64)
+    for j in range(tab.shape[0]):
+        for t in tab[j]:
+            if t >= 0:
+                blk_of[t] = j
+    mask = np.zeros((g.B, g.Hd, g.n_tot, g.n_tot), dtype=bool)
+    for b in range(g.B):
+        for h in range(g.Hd):
+            for qb in range(g.nb):
+                keys = np.concatenate([tab[j][tab[j] >= 0] for j in idx[b, h, qb, :cnt[b, h, qb]]])
+                qs = tab[qb][tab[qb] >= 0]
+                mask[b, h, np.ix_(qs, keys)[0], np.ix_(qs, keys)[1]] = True
+            for qb in range(g.nb, g.nb + g.nb_text):
+                qs = tab[qb][tab[qb] >= 0]
+                mask[b, h, qs, :] = True
+    return mask
+
+
+def sdpa(q, k, v, mask=None):
+    """torch fp64 scaled-dot-product attention in the original layout."""
+    tq = torch.from_numpy(np.asarray(q, np.float64)).permute(0, 2, 1, 3)
+    tk = torch.from_numpy(np.asarray(k, np.float64)).permute(0, 2, 1, 3)
+    tv = torch.from_numpy(np.asarray(v, np.float64)).permute(0, 2, 1, 3)
+    m = None if mask is None else torch.from_numpy(mask)
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=m)
+    return o.permute(0, 2, 1, 3).numpy()
+
+
+def random_lists(g, seed, max_blocks=None):
+    """Random ascending lists of distinct video blocks + all text blocks."""
+    rng = np.random.default_rng(seed)
+    kmax = g.nb + g.nb_text
+    idx = np.full((g.B, g.Hd, g.nb, kmax), -1, dtype=np.int32)
+    cnt = np.zeros((g.B, g.Hd, g.nb), dtype=np.int32)
+    for b in range(g.B):
+        for h in range(g.Hd):
+            for i in range(g.nb):
+                m = rng.integers(1, (max_blocks or g.nb) + 1)
+                sel = np.sort(rng.choice(g.nb, size=m, replace=False))
+                lst = list(sel) + list(range(g.nb, g.nb + g.nb_text))
+                idx[b, h, i, :len(lst)] = lst
+                cnt[b, h, i] = len(lst)
+    return idx, cnt
+
+
+RAGGED = dict(B=2, T=3, H=5, W=7, bf=2, br=4, bc=4, Hd=2, D=16, n_text=5)
+EVEN = dict(B=1, T=4, H=8, W=8, bf=2, br=4, bc=4, Hd=2, D=8, n_text=0)
+
+
+# ------------------------------------------------------------ layout pins --
+@pytest.mark.parametrize("geo", [EVEN, RAGGED, dict(B=1, T=5, H=9, W=6, bf=1, br=8, bc=16,
+                                                    Hd=3, D=8, n_text=130)])
+def test_permute_matches_reshape_layout(geo):
+    g = orc.Geometry(**geo)
+    x = rand_x(g, 1)
+    tab = token_table(g).reshape(-1)
+    expect = np.zeros((g.B, g.Hd, g.npad_tot, g.D))
+    valid = tab >= 0
+    expect[:, :, valid, :] = x[:, tab[valid], :, :].transpose(0, 2, 1, 3)
+    got = orc.permute(g, x)
+    assert np.array_equal(got, expect)
+    # every valid token appears exactly once; pads are exactly zero
+    assert np.array_equal(np.sort(tab[valid]), np.arange(g.n_tot))
+    assert np.all(got[:, :, ~valid, :] == 0)
+
+
+@pytest.mark.parametrize("geo", [EVEN, RAGGED])
+def test_unpermute_inverts_permute(geo):
+    g = orc.Geometry(**geo)
+    x = rand_x(g, 2)
+    assert np.array_equal(orc.unpermute(g, orc.permute(g, x)), x.astype(np.float64))
+
+
+def test_permute_dense_even_grid_is_pure_transpose():
+    # 1x1x1 blocks: the blocked layout is just [B, Hd, N, D]
+    g = orc.Geometry(B=1, T=2, H=3, W=4, bf=1, br=1, bc=1, Hd=2, D=4, n_text=3)
+    x = rand_x(g, 3)
+    assert np.array_equal(orc.permute(g, x), x.transpose(0, 2, 1, 3).astype(np.float64))
+
+
+# ----------------------------------------------------------- centroid pin --
+@pytest.mark.parametrize("geo", [EVEN, RAGGED])
+def test_centroids_are_means_over_valid_tokens(geo):
+    g = orc.Geometry(**geo)
+    x = rand_x(g, 4)
+    Tp, Hp, Wp = g.nbt * g.bf, g.nby * g.br, g.nbx * g.bc
+    grid = np.full((g.B, Tp, Hp, Wp, g.Hd, g.D), np.nan)
+    grid[:, :g.T, :g.H, :g.W] = x[:, :g.n_video].reshape(g.B, g.T, g.H, g.W, g.Hd, g.D)
+    blk = grid.reshape(g.B, g.nbt, g.bf, g.nby, g.br, g.nbx, g.bc, g.Hd, g.D)
+    expect = np.nanmean(blk, axis=(2, 4, 6)).reshape(g.B, g.nb, g.Hd, g.D).transpose(0, 2, 1, 3)
+    np.testing.assert_allclose(orc.centroids(g, x), expect, rtol=0, atol=1e-12)
+
+
+# -------------------------------------------------------------- score pin --
+def test_scores_are_row_softmax_of_scaled_dots():
+    g = orc.Geometry(**RAGGED)
+    rng = np.random.default_rng(5)
+    qc = rng.standard_normal((g.B, g.Hd, g.nb, g.D))
+    kc = rng.standard_normal((g.B, g.Hd, g.nb, g.D))
+    expect = scipy.special.softmax(np.einsum("bhid,bhjd->bhij", qc, kc) / math.sqrt(g.D), axis=-1)
+    got = orc.scores(g, qc, kc)
+    np.testing.assert_allclose(got, expect, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(got.sum(-1), 1.0, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------- selection pins --
+def _golden_k_table():
+    rows = []
+    with open(os.path.join(GOLDEN, "k_for_density.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if line:
+                rho, nb, k = line.split()
+                rows.append((float(rho), int(nb), int(k)))
+    return rows
+
+
+def test_k_for_density_golden():
+    rows = _golden_k_table()
+    assert len(rows) >= 9
+    for rho, nb, k in rows:
+        assert orc.k_for_density(rho, nb) == k, (rho, nb, k)
+
+
+def _rand_p(g, seed, spread=2.0):
+    rng = np.random.default_rng(seed)
+    s = rng.standard_normal((g.B, g.Hd, g.nb, g.nb)) * spread
+    return scipy.special.softmax(s, axis=-1)
+
+
+@pytest.mark.parametrize("rho", [0.125, 0.25, 0.5, 0.75, 1.0])
+def test_topk_is_max_mass_subset(rho):
+    g = orc.Geometry(**RAGGED)          # nb = 8, one text block
+    p = _rand_p(g, 6)
+    idx, cnt, tie = orc.select(g, p, 0, [rho] * g.Hd)
+    k = orc.k_for_density(rho, g.nb)
+    assert np.all(cnt == k + g.nb_text)
+    for b, h, i in itertools.product(range(g.B), range(g.Hd), range(g.nb)):
+        best = max(itertools.combinations(range(g.nb), k), key=lambda s: p[b, h, i, list(s)].sum())
+        lst = list(idx[b, h, i, :cnt[b, h, i]])
+        assert lst == sorted(best) + list(range(g.nb, g.nb + g.nb_text))
+        assert tie[b, h, i] == 0
+
+
+@pytest.mark.parametrize("tau", [0.3, 0.5, 0.9, 0.99, 1.0])
+def test_topp_is_shortest_prefix_reaching_tau(tau):
+    g = orc.Geometry(**RAGGED)
+    p = _rand_p(g, 7)
+    idx, cnt, tie = orc.select(g, p, 1, [tau] * g.Hd)
+    for b, h, i in itertools.product(range(g.B), range(g.Hd), range(g.nb)):
+        if tie[b, h, i]:
+            continue
+        row = p[b, h, i]
+        for m in range(1, g.nb + 1):
+            best = max(itertools.combinations(range(g.nb), m), key=lambda s: row[list(s)].sum())
+            if row[list(best)].sum() >= tau:
+                break
+        lst = list(idx[b, h, i, :cnt[b, h, i]])
+        assert lst == sorted(best) + list(range(g.nb, g.nb + g.nb_text)), (b, h, i)
+
+
+def test_topk_ties_break_by_lower_index_and_are_reported():
+    g = orc.Geometry(B=1, T=1, H=1, W=8, bf=1, br=1, bc=1, Hd=1, D=4, n_text=0)
+    p = np.full((1, 1, 8, 8), 1 / 8.0)
+    idx, cnt, tie = orc.select(g, p, 0, [0.25])
+    assert np.all(idx[0, 0, :, :2] == [0, 1]) and np.all(tie == 1)
+
+
+def test_topp_tie_flag_near_threshold():
+    g = orc.Geometry(B=1, T=1, H=1, W=4, bf=1, br=1, bc=1, Hd=1, D=4, n_text=0)
+    p = np.tile(np.array([0.5, 0.3, 0.15, 0.05]), (1, 1, 4, 1))
+    _, cnt, tie = orc.select(g, p, 1, [0.8])
+    assert np.all(cnt == 2) and np.all(tie == 1)          # 0.5 + 0.3 == tau
+    _, cnt, tie = orc.select(g, p, 1, [0.7])
+    assert np.all(cnt == 2) and np.all(tie == 0)
+
+
+# ---------------------------------------------------------- attention pins --
+def test_density_one_equals_dense_attention():
+    g = orc.Geometry(**RAGGED)
+    q, k, v = rand_x(g, 8), rand_x(g, 9), rand_x(g, 10)
+    idx = np.tile(np.arange(g.nb + g.nb_text, dtype=np.int32), (g.B, g.Hd, g.nb, 1))
+    cnt = np.full((g.B, g.Hd, g.nb), g.nb + g.nb_text, dtype=np.int32)
+    np.testing.assert_allclose(orc.attention(g, q, k, v, idx, cnt), sdpa(q, k, v),
+                               rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("geo", [RAGGED, dict(B=1, T=5, H=9, W=6, bf=1, br=8, bc=16, Hd=2, D=8,
+                                             n_text=130)])
+def test_sparse_attention_equals_masked_sdpa(geo):
+    g = orc.Geometry(**geo)
+    q, k, v = rand_x(g, 11), rand_x(g, 12), rand_x(g, 13)
+    idx, cnt = random_lists(g, 14)
+    got = orc.attention(g, q, k, v, idx, cnt)
+    np.testing.assert_allclose(got, sdpa(q, k, v, token_mask(g, idx, cnt)), rtol=1e-11, atol=1e-12)
+
+
+def test_forward_pipeline_equals_masked_sdpa():
+    g = orc.Geometry(**RAGGED)
+    q, k, v = rand_x(g, 15), rand_x(g, 16), rand_x(g, 17)
+    o, idx, cnt, tie, p = orc.forward(g, q, k, v, 0, [0.25] * g.Hd)
+    assert np.all(cnt == 2 + g.nb_text)
+    np.testing.assert_allclose(o, sdpa(q, k, v, token_mask(g, idx, cnt)), rtol=1e-11, atol=1e-12)
+
+
+def test_ones_values_give_ones():
+    g = orc.Geometry(**RAGGED)
+    q, k = rand_x(g, 18), rand_x(g, 19)
+    v = np.ones((g.B, g.n_tot, g.Hd, g.D), dtype=np.float32)
+    idx, cnt = random_lists(g, 20)
+    np.testing.assert_allclose(orc.attention(g, q, k, v, idx, cnt), 1.0, rtol=0, atol=1e-13)
+
+
+def test_equal_keys_give_plain_mean_of_allowed_values():
+    g = orc.Geometry(**RAGGED)
+    q, v = rand_x(g, 21), rand_x(g, 22)
+    k = np.ones((g.B, g.n_tot, g.Hd, g.D), dtype=np.float32)
+    idx, cnt = random_lists(g, 23)
+    m = token_mask(g, idx, cnt).astype(np.float64)                 # [B,Hd,Nq,Nk]
+    expect = np.einsum("bhqk,bkhd->bqhd", m, v.astype(np.float64)) / m.sum(-1).transpose(0, 2, 1)[..., None]
+    np.testing.assert_allclose(orc.attention(g, q, k, v, idx, cnt), expect, rtol=1e-12, atol=1e-13)
+
+
+def test_row_subset_matches_full_output():
+    g = orc.Geometry(**RAGGED)
+    q, k, v = rand_x(g, 24), rand_x(g, 25), rand_x(g, 26)
+    idx, cnt = random_lists(g, 27)
+    full = orc.attention(g, q, k, v, idx, cnt)
+    rows = np.array([0, 7, 33, g.n_video - 1, g.n_video, g.n_tot - 1])
+    np.testing.assert_array_equal(orc.attention(g, q, k, v, idx, cnt, rows=rows), full[:, rows])
+
+
+def test_selected_pairs_counts_mask_entries():
+    g = orc.Geometry(**RAGGED)
+    idx, cnt = random_lists(g, 28)
+    assert orc.selected_pairs(g, idx, cnt) == int(token_mask(g, idx, cnt).sum())
