@@ -1,0 +1,434 @@
+"""Benchmark of the block-sparse attention executor on one node.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one bsa_forward (permute -> select -> attention -> unpermute) over
+one batch of synthetic input already resident in HBM.  Default workload: the
+HunyuanVideo 720p 61-frame shape (16x45x80 latent grid + 256 text tokens,
+24 heads, head_dim 128, bf16, 1x8x16 blocks, density 0.15).
+
+Printed: one JSON line on rank 0.  value = effective TFLOP/s of the whole job
+= 4 x selected valid (query, key) pairs x head_dim (summed over heads and
+ranks) / max-over-ranks device time.  Per-phase times come from a second loop
+that issues the same four calls separately, with CUDA events on the
+launching stream.  Under torchrun every rank runs its own replica of the
+workload (weak scaling, no collective on the data path).
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+METRIC = "sparse-attn ms/call + effective TFLOP/s (% bf16 TC peak), 57.6k-token shape"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d.get("bf16_tflops_sustained", d.get("bf16_tflops")), d.get("hbm_gbs"), "measured"
+    return 1400.0, 6650.0, "fallback"
+
+
+def attn_source_sha() -> str:
+    h = hashlib.sha256()
+    for name in ("attn.cu", "common.cuh", "kernels.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_attention_permute_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was
+    captured on the current attention source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"attn_tc_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if line.startswith("bench_key:"):
+                k, _, v = line[len("bench_key:"):].strip().partition("=")
+                vals[k.strip()] = v.strip()
+    if vals.get("attn_source_sha") != attn_source_sha():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def reduce_max(vals, device="cpu"):
+    """Element-wise max of per-rank values over all ranks (identity on one rank)."""
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_tflops(world: int, flops_per_rank_step: float, step_ms: float) -> float:
+    """Whole-job throughput: every rank processes one replica per step."""
+    return world * flops_per_rank_step / (step_ms * 1e-3) / 1e12
+
+
+def effective_pairs(plan, idx, cnt) -> int:
+    """Selected valid (query, key) token pairs, summed over batch and heads."""
+    i = plan.info
+    nbk = i.nb + i.nb_text
+    valid = np.zeros(nbk, dtype=np.int64)
+    for j in range(i.nb):
+        tb, yb, xb = j // (i.nby * i.nbx), (j // i.nbx) % i.nby, j % i.nbx
+        valid[j] = (min(i.bf, i.T - tb * i.bf) * min(i.br, i.H - yb * i.br)
+                    * min(i.bc, i.W - xb * i.bc))
+    for t in range(i.nb_text):
+        valid[i.nb + t] = min(i.bs, i.n_text - t * i.bs)
+    vd = torch.from_numpy(valid).to(idx.device)
+    kmax = idx.shape[-1]
+    ar = torch.arange(kmax, device=idx.device)
+    sel = (ar[None, None, None, :] < cnt[..., None])
+    keys = torch.where(sel, vd[idx.clamp(0, nbk - 1).long()], torch.zeros_like(idx, dtype=torch.long))
+    keys_per_row = keys.sum(-1)                                  # [B,Hd,nb]
+    video = int((keys_per_row * vd[:i.nb][None, None, :]).sum())
+    text = int(valid[i.nb:].sum()) * i.n_tot * i.batch * i.heads
+    return video + text
+
+
+def run_ours(args, rank, world, local):
+    import block_sparse_attention_permute_b200 as bsa
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=dev)
+    w = synthetic.workload(args.workload)
+    q, k, v = synthetic.make_qkv(w)
+    plan = bsa.plan_for(w, dev)
+    kmax = plan.kmax_for(w.mode, w.params)
+    sel_ws, fwd_ws = plan.workspace_size(kmax)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    out = torch.empty_like(qd)
+    ws = torch.empty(fwd_ws, dtype=torch.uint8, device=dev)
+    idx = torch.empty((w.B, w.Hd, plan.info.nb, kmax), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.B, w.Hd, plan.info.nb), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    L = bsa.load()
+    params = bsa._params(w.params, w.Hd)
+    P = bsa._ptr
+
+    def forward():
+        bsa._check(L.bsa_forward(plan._h, P(qd), P(kd), P(vd), w.mode, params, kmax, P(out), P(idx),
+                                 P(cnt), P(ws), ws.numel(), None, bsa._stream(dev)))
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        forward()
+    plan.check_status()
+    pairs = effective_pairs(plan, idx, cnt)
+    flops = 4.0 * pairs * w.D
+
+    # ---- main timed loop: K whole steps
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            forward()
+        ev1.record(stream)
+        barrier()
+    plan.check_status()
+    step_ms = ev0.elapsed_time(ev1) / args.steps
+    clocks = clk.summary()
+
+    # ---- phase loop: the same four calls, separately timed
+    qb, kb, vb, ob = (torch.empty(plan.blk_shape, dtype=plan.dtype, device=dev) for _ in range(4))
+    qc, kc = (torch.empty(plan.cent_shape, dtype=torch.float32, device=dev) for _ in range(2))
+    names = ["permute", "select", "attention", "unpermute"]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    calls = [
+        lambda: L.bsa_permute_qkv(plan._h, P(qd), P(kd), P(vd), P(qb), P(kb), P(vb), P(qc), P(kc),
+                                  bsa._stream(dev)),
+        lambda: L.bsa_select_centroids(plan._h, P(qc), P(kc), w.mode, params, kmax, P(idx), P(cnt),
+                                       None, bsa._stream(dev)),
+        lambda: L.bsa_attention(plan._h, P(qb), P(kb), P(vb), P(idx), P(cnt), kmax, P(ob), None,
+                                bsa._stream(dev)),
+        lambda: L.bsa_unpermute(plan._h, P(ob), P(out), bsa._stream(dev)),
+    ]
+    for _ in range(args.warmup):
+        for c in calls:
+            bsa._check(c())
+    barrier()
+    for s in range(args.steps):
+        evs[s][0].record(stream)
+        for ci, c in enumerate(calls):
+            bsa._check(c())
+            evs[s][ci + 1].record(stream)
+    barrier()
+    plan.check_status()
+    phase_ms = {n: sum(evs[s][ci].elapsed_time(evs[s][ci + 1]) for s in range(args.steps)) / args.steps
+                for ci, n in enumerate(names)}
+
+    # ---- end to end: pinned host buffers, copies inside the timed region
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    for _ in range(2):
+        qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
+        forward()
+        oh.copy_(out, non_blocking=True)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
+        forward()
+        oh.copy_(out, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    h2d = 3 * q.numel() * q.element_size()
+    d2h = q.numel() * q.element_size()
+
+    step_ms, e2e_ms, attn_ms = reduce_max([step_ms, e2e_ms, phase_ms["attention"]], dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+    if rank != 0:
+        return
+    peak_tf, hbm_gbs, peak_src = peaks()
+    value = job_tflops(world, flops, step_ms)
+    attn_tf = flops / (attn_ms * 1e-3) / 1e12
+    traffic = profiled_traffic(args.workload)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": w.name,
+            "shape": f"grid {w.T}x{w.H}x{w.W} + {w.n_text} text, block {w.bf}x{w.br}x{w.bc}, "
+                     f"{w.Hd} heads, head_dim {w.D}, batch {w.B}",
+            "selection": ("top-k density " if w.mode == 0 else "top-p tau ") +
+                         (str(w.params[0]) if len(set(w.params)) == 1 else "per-head mix"),
+            "parallelism": f"replicas x{world} (no collective)",
+            "l2": f"inputs {3 * q.numel() * q.element_size() / 1e9:.2f} GB > 126 MB L2 (no flush)",
+            "effective_tflop_per_step": round(flops / 1e12, 4),
+            "selected_pairs": pairs,
+        },
+        "phases_ms": {n: round(t, 4) for n, t in phase_ms.items()},
+        "attn_tflops": round(attn_tf, 2),
+        "attn_frac_of_peak": round(attn_tf / peak_tf, 4),
+        "permute_select_share_of_attn": round(
+            (phase_ms["permute"] + phase_ms["select"]) / phase_ms["attention"], 4),
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "attn_tc_kernel",
+            "achieved": round(attn_tf, 2),
+            "peak": peak_tf,
+            "peak_source": f"{peak_src} bf16_tflops_sustained (MEASURED_PEAKS.json)",
+            "unit": "TFLOP/s",
+            "frac": round(attn_tf / peak_tf, 4),
+            "traffic": traffic,
+        },
+        "e2e": {"value": round(job_tflops(world, flops, e2e_ms), 2), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, q, k, v, budget_s=args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(w, q, k, v, budget_s=20.0):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload."""
+    import oracle as orc
+    g = orc.Geometry(*w.geometry_args())
+    qn, kn, vn = (t.float().numpy() for t in (q, k, v))
+    t0 = time.perf_counter()
+    p = orc.scores(g, orc.centroids(g, qn), orc.centroids(g, kn))
+    idx, cnt, _ = orc.select(g, p, w.mode, w.params)
+    t_sel = time.perf_counter() - t0
+    # attention on whole query blocks (all heads), as many as fit the budget
+    rng = np.random.default_rng(0)
+    order = rng.permutation(g.nb)
+    done_rows, pairs, t_att, nblk = [], 0, 0.0, 0
+    valid_tab = {}
+    for j in order:
+        tb, yb, xb = j // (g.nby * g.nbx), (j // g.nbx) % g.nby, j % g.nbx
+        rows = [(t * g.H + y) * g.W + x
+                for t in range(tb * g.bf, min(g.T, (tb + 1) * g.bf))
+                for y in range(yb * g.br, min(g.H, (yb + 1) * g.br))
+                for x in range(xb * g.bc, min(g.W, (xb + 1) * g.bc))]
+        t1 = time.perf_counter()
+        orc.attention(g, qn, kn, vn, idx, cnt, rows=np.array(rows))
+        t_att += time.perf_counter() - t1
+        nblk += 1
+        for b in range(g.B):
+            for h in range(g.Hd):
+                keys = 0
+                for jj in idx[b, h, j, :cnt[b, h, j]]:
+                    if jj not in valid_tab:
+                        valid_tab[jj] = _valid_count(g, int(jj))
+                    keys += valid_tab[jj]
+                pairs += keys * len(rows)
+        if t_att + t_sel >= budget_s:
+            break
+    flops = 4.0 * pairs * g.D
+    tf = flops / t_att / 1e12
+    return {"value": tf, "unit": "TFLOP/s", "cores": orc.threads(), "kind": "oracle",
+            "sample": f"oracle centroids+scores+selection on the full workload ({t_sel:.1f} s), "
+                      f"attention on {nblk} random query blocks x all {g.Hd} heads "
+                      f"({t_att:.1f} s); value = effective FLOP of the sampled attention / its time"}
+
+
+def _valid_count(g, j):
+    if j >= g.nb:
+        return min(g.bs, g.n_text - (j - g.nb) * g.bs)
+    tb, yb, xb = j // (g.nby * g.nbx), (j // g.nbx) % g.nby, j % g.nbx
+    return (min(g.bf, g.T - tb * g.bf) * min(g.br, g.H - yb * g.br) * min(g.bc, g.W - xb * g.bc))
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = synthetic.workload(args.workload)
+    q, k, v = synthetic.make_qkv(w)
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    vals = []
+    for s in range(args.warmup + args.steps):
+        cb = cpu_baseline(w, q, k, v, budget_s=per_step)
+        if s >= args.warmup:
+            vals.append(cb["value"])
+    value = float(np.mean(vals))
+    cb["value"] = value
+    line = {
+        "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": w.name, "parallelism": "host cores (oracle threads)"},
+        "cpu_baseline": cb,
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="hunyuan", choices=synthetic.WORKLOADS)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,264 @@
+"""Python binding of libbsa — 3D block-sparse attention for video DiTs on B200.
+
+Argument marshalling only: every step runs in the CUDA kernels of
+``libbsa.so`` (built in-tree by ``python -m block_sparse_attention_permute_b200.build``).
+There is no fallback: importing works without the library, but every call
+raises ``BsaError`` if ``libbsa.so`` is missing or the tensors are not on a
+CUDA device.  PyTorch provides device memory and streams.
+
+The calls mirror include/bsa.h (SPADE §3.3 "Head-wise Sparse Attention"):
+``Plan.permute``/``unpermute`` (blocked layout), ``Plan.select`` (centroid
+scores and Top-K / Top-P), ``Plan.attention`` (flash block-sparse attention)
+and ``Plan.forward`` (all four in sequence).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["Plan", "BsaError", "TOPK", "TOPP", "lib_path", "load"]
+
+TOPK = 0
+TOPP = 1
+_DT = {torch.float32: 0, torch.bfloat16: 1}
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libbsa.so")
+_lib = None
+
+
+class BsaError(RuntimeError):
+    """A libbsa call returned an error status (or the library is unavailable)."""
+
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"libbsa status {status}: {msg}")
+        self.status = status
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in
+                ("batch", "T", "H", "W", "bf", "br", "bc", "heads", "head_dim", "n_text", "dtype",
+                 "Tp", "Hp", "Wp", "nbt", "nby", "nbx", "nb", "nb_text", "bs")] + \
+               [("n_video", ctypes.c_longlong), ("n_tot", ctypes.c_longlong),
+                ("npad_tot", ctypes.c_longlong), ("attn_path", ctypes.c_int)]
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load libbsa.so (raises BsaError if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise BsaError(-1, f"{_LIB_PATH} is missing; build it with "
+                           "`python -m block_sparse_attention_permute_b200.build`")
+    L = ctypes.CDLL(_LIB_PATH)
+    P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.bsa_last_error_string.restype = ctypes.c_char_p
+    L.bsa_version.restype = I
+    sigs = {
+        "bsa_plan_create": [ctypes.POINTER(P)] + [I] * 11,
+        "bsa_plan_destroy": [P],
+        "bsa_plan_get_info": [P, ctypes.POINTER(PlanInfo)],
+        "bsa_kmax_for": [P, I, P, ctypes.POINTER(I)],
+        "bsa_workspace_size": [P, I, ctypes.POINTER(Z), ctypes.POINTER(Z)],
+        "bsa_permute": [P, P, P, P, P],
+        "bsa_permute_qkv": [P] * 10,
+        "bsa_unpermute": [P, P, P, P],
+        "bsa_select": [P, P, P, I, P, I, P, P, P, P, Z, P],
+        "bsa_select_centroids": [P, P, P, I, P, I, P, P, P, P],
+        "bsa_attention": [P, P, P, P, P, P, I, P, P, P],
+        "bsa_forward": [P, P, P, P, I, P, I, P, P, P, P, Z, P, P],
+        "bsa_check_status": [P, P],
+    }
+    for name, args in sigs.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = I
+    _lib = L
+    return L
+
+
+def _check(status: int):
+    if status != 0:
+        raise BsaError(status, load().bsa_last_error_string().decode())
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _params(p, heads):
+    if isinstance(p, (int, float)):
+        p = [float(p)] * heads
+    arr = (ctypes.c_double * heads)(*[float(x) for x in p])
+    if len(p) != heads:
+        raise BsaError(1, f"expected {heads} per-head parameters, got {len(p)}")
+    return arr
+
+
+class Plan:
+    """One attention problem: grid (T,H,W), block (bf,br,bc), heads, head_dim, text tokens."""
+
+    def __init__(self, batch, T, H, W, bf, br, bc, heads, head_dim, n_text=0,
+                 dtype=torch.bfloat16, device=None):
+        L = load()
+        if dtype not in _DT:
+            raise BsaError(1, f"dtype must be float32 or bfloat16, got {dtype}")
+        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None \
+            else torch.device(device)
+        if self.device.type != "cuda":
+            raise BsaError(1, "libbsa runs on CUDA devices only")
+        self.dtype = dtype
+        self._h = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            _check(L.bsa_plan_create(ctypes.byref(self._h), batch, T, H, W, bf, br, bc, heads,
+                                     head_dim, n_text, _DT[dtype]))
+        info = PlanInfo()
+        _check(L.bsa_plan_get_info(self._h, ctypes.byref(info)))
+        self.info = info
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h and _lib is not None:
+            try:
+                with torch.cuda.device(self.device):
+                    _lib.bsa_plan_destroy(h)
+            except Exception:
+                pass
+            self._h = None
+
+    # ---------------------------------------------------------------- sizes
+    @property
+    def orig_shape(self):
+        i = self.info
+        return (i.batch, i.n_tot, i.heads, i.head_dim)
+
+    @property
+    def blk_shape(self):
+        i = self.info
+        return (i.batch, i.heads, i.npad_tot, i.head_dim)
+
+    @property
+    def cent_shape(self):
+        i = self.info
+        return (i.batch, i.heads, i.nb, i.head_dim)
+
+    def kmax_for(self, mode, params) -> int:
+        k = ctypes.c_int()
+        _check(load().bsa_kmax_for(self._h, mode, _params(params, self.info.heads), ctypes.byref(k)))
+        return k.value
+
+    def workspace_size(self, kmax):
+        a, b = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(load().bsa_workspace_size(self._h, kmax, ctypes.byref(a), ctypes.byref(b)))
+        return a.value, b.value
+
+    def _new(self, shape, dtype=None):
+        return torch.empty(shape, dtype=dtype or self.dtype, device=self.device)
+
+    def _check_tensor(self, t, shape, dtype=None, name="tensor"):
+        dtype = dtype or self.dtype
+        if not isinstance(t, torch.Tensor) or t.device != self.device:
+            raise BsaError(1, f"{name} must be a tensor on {self.device}")
+        if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+            raise BsaError(1, f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}, "
+                              f"got {t.dtype} {tuple(t.shape)}")
+
+    # ---------------------------------------------------------------- calls
+    def permute(self, x, centroids=False, out=None):
+        self._check_tensor(x, self.orig_shape, name="x")
+        out = self._new(self.blk_shape) if out is None else out
+        cent = self._new(self.cent_shape, torch.float32) if centroids else None
+        _check(load().bsa_permute(self._h, _ptr(x), _ptr(out), _ptr(cent), _stream(self.device)))
+        return (out, cent) if centroids else out
+
+    def permute_qkv(self, q, k, v):
+        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+            self._check_tensor(t, self.orig_shape, name=n)
+        qb, kb, vb = (self._new(self.blk_shape) for _ in range(3))
+        qc, kc = (self._new(self.cent_shape, torch.float32) for _ in range(2))
+        _check(load().bsa_permute_qkv(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(qb), _ptr(kb),
+                                      _ptr(vb), _ptr(qc), _ptr(kc), _stream(self.device)))
+        return qb, kb, vb, qc, kc
+
+    def unpermute(self, o_blk, out=None):
+        self._check_tensor(o_blk, self.blk_shape, name="o_blk")
+        out = self._new(self.orig_shape) if out is None else out
+        _check(load().bsa_unpermute(self._h, _ptr(o_blk), _ptr(out), _stream(self.device)))
+        return out
+
+    def _lists(self, kmax):
+        i = self.info
+        return (self._new((i.batch, i.heads, i.nb, kmax), torch.int32),
+                self._new((i.batch, i.heads, i.nb), torch.int32))
+
+    def select(self, q_blk, k_blk, mode, params, kmax=None, scores=False):
+        self._check_tensor(q_blk, self.blk_shape, name="q_blk")
+        self._check_tensor(k_blk, self.blk_shape, name="k_blk")
+        kmax = self.kmax_for(mode, params) if kmax is None else kmax
+        idx, cnt = self._lists(kmax)
+        i = self.info
+        sc = self._new((i.batch, i.heads, i.nb, i.nb), torch.float32) if scores else None
+        ws = self._new((max(self.workspace_size(kmax)[0], 1),), torch.uint8)
+        _check(load().bsa_select(self._h, _ptr(q_blk), _ptr(k_blk), mode,
+                                 _params(params, i.heads), kmax, _ptr(idx), _ptr(cnt), _ptr(sc),
+                                 _ptr(ws), ws.numel(), _stream(self.device)))
+        return (idx, cnt, sc) if scores else (idx, cnt)
+
+    def select_centroids(self, q_cent, k_cent, mode, params, kmax=None, scores=False):
+        self._check_tensor(q_cent, self.cent_shape, torch.float32, "q_cent")
+        self._check_tensor(k_cent, self.cent_shape, torch.float32, "k_cent")
+        kmax = self.kmax_for(mode, params) if kmax is None else kmax
+        idx, cnt = self._lists(kmax)
+        i = self.info
+        sc = self._new((i.batch, i.heads, i.nb, i.nb), torch.float32) if scores else None
+        _check(load().bsa_select_centroids(self._h, _ptr(q_cent), _ptr(k_cent), mode,
+                                           _params(params, i.heads), kmax, _ptr(idx), _ptr(cnt),
+                                           _ptr(sc), _stream(self.device)))
+        return (idx, cnt, sc) if scores else (idx, cnt)
+
+    def attention(self, q_blk, k_blk, v_blk, idx, cnt, out=None, dev_status=None):
+        for t, n in ((q_blk, "q_blk"), (k_blk, "k_blk"), (v_blk, "v_blk")):
+            self._check_tensor(t, self.blk_shape, name=n)
+        i = self.info
+        kmax = idx.shape[-1]
+        self._check_tensor(idx, (i.batch, i.heads, i.nb, kmax), torch.int32, "idx")
+        self._check_tensor(cnt, (i.batch, i.heads, i.nb), torch.int32, "cnt")
+        out = self._new(self.blk_shape) if out is None else out
+        _check(load().bsa_attention(self._h, _ptr(q_blk), _ptr(k_blk), _ptr(v_blk), _ptr(idx),
+                                    _ptr(cnt), kmax, _ptr(out), _ptr(dev_status),
+                                    _stream(self.device)))
+        return out
+
+    def forward(self, q, k, v, mode, params, kmax=None, out=None, workspace=None,
+                return_lists=False):
+        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+            self._check_tensor(t, self.orig_shape, name=n)
+        kmax = self.kmax_for(mode, params) if kmax is None else kmax
+        out = self._new(self.orig_shape) if out is None else out
+        need = self.workspace_size(kmax)[1]
+        ws = self._new((need,), torch.uint8) if workspace is None else workspace
+        idx, cnt = self._lists(kmax) if return_lists else (None, None)
+        _check(load().bsa_forward(self._h, _ptr(q), _ptr(k), _ptr(v), mode,
+                                  _params(params, self.info.heads), kmax, _ptr(out), _ptr(idx),
+                                  _ptr(cnt), _ptr(ws), ws.numel(), None, _stream(self.device)))
+        return (out, idx, cnt) if return_lists else out
+
+    def check_status(self):
+        """Synchronise the current stream and raise if a kernel recorded an error."""
+        _check(load().bsa_check_status(self._h, _stream(self.device)))
+
+
+def plan_for(w, device=None) -> Plan:
+    """A Plan for a synthetic Workload-like object (attributes B,T,H,W,bf,br,bc,Hd,D,n_text,dtype)."""
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    return Plan(w.B, w.T, w.H, w.W, w.bf, w.br, w.bc, w.Hd, w.D, w.n_text, dt, device)

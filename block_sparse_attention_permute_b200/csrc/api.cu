@@ -1,0 +1,413 @@
+// api.cu — the C ABI of libbsa (declared in include/bsa.h): argument
+// validation, plan state, workspace carving, TMA tensor maps and launches.
+// Every entry point validates on the host before it launches anything.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "bsa.h"
+#include "kernels.cuh"
+
+struct bsa_plan_s {
+  Geo g;
+  bsa_dtype dtype;
+  int device;
+  int attn_path;        // 1 tcgen05, 0 SIMT
+  int32_t* d_status;    // device status word
+  uint32_t* d_masks;    // [(nb + nb_text) * 4] slot validity bits (bs == 128)
+};
+
+namespace {
+
+thread_local std::string g_err;
+
+bsa_status fail(bsa_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+bsa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(BSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t elem_size(const bsa_plan_s* p) { return p->dtype == BSA_BF16 ? 2 : 4; }
+
+size_t blk_bytes(const bsa_plan_s* p) {
+  return (size_t)p->g.B * p->g.Hd * p->g.npad_tot * p->g.D * elem_size(p);
+}
+size_t cent_bytes(const bsa_plan_s* p) {
+  return (size_t)p->g.B * p->g.Hd * p->g.nb * p->g.D * sizeof(float);
+}
+
+// k per head for a density (the fraction of key blocks each query block keeps).
+int k_for_density(double rho, int nb) {
+  long long k = (long long)std::ceil(rho * (double)nb - 1e-9);
+  if (k < 1) k = 1;
+  if (k > nb) k = nb;
+  return (int)k;
+}
+
+bsa_status check_params(const bsa_plan_s* p, bsa_select_mode mode, const double* param,
+                        int* kmax_needed) {
+  if (param == nullptr) return fail(BSA_ERR_INVALID_ARG, "param_per_head is NULL");
+  if (mode != BSA_TOPK && mode != BSA_TOPP) return fail(BSA_ERR_INVALID_ARG, "bad select mode %d", (int)mode);
+  int kmax = 0;
+  for (int h = 0; h < p->g.Hd; ++h) {
+    const double v = param[h];
+    if (!(v > 0.0 && v <= 1.0))
+      return fail(BSA_ERR_INVALID_ARG, "%s of head %d is %g, must be in (0, 1]",
+                  mode == BSA_TOPK ? "density" : "tau", h, v);
+    const int k = mode == BSA_TOPK ? k_for_density(v, p->g.nb) : p->g.nb;
+    if (k > kmax) kmax = k;
+  }
+  *kmax_needed = kmax + p->g.nb_text;
+  return BSA_OK;
+}
+
+bsa_status check_plan(const bsa_plan_s* p) {
+  if (p == nullptr) return fail(BSA_ERR_INVALID_ARG, "plan is NULL");
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev != p->device)
+    return fail(BSA_ERR_INVALID_ARG, "plan was created on device %d, current device is %d", p->device, dev);
+  return BSA_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2D map over a blocked bf16 tensor: rows x D, box 64 x 128, 128-byte swizzle.
+bsa_status make_tile_map(CUtensorMap* m, const void* base, long long rows, int D) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return BSA_OK;
+}
+
+bsa_status run_select(const bsa_plan_s* p, const float* qc, const float* kc, bsa_select_mode mode,
+                      const double* param, int kmax, int32_t* idx, int32_t* cnt, float* scores,
+                      cudaStream_t st) {
+  int need = 0;
+  bsa_status s = check_params(p, mode, param, &need);
+  if (s != BSA_OK) return s;
+  if (kmax < need) return fail(BSA_ERR_INVALID_ARG, "kmax %d is below the %d entries a list can need", kmax, need);
+  if (p->g.nb == 0) return BSA_OK;
+  if (!qc || !kc || !idx || !cnt) return fail(BSA_ERR_INVALID_ARG, "NULL centroid or list pointer");
+  if (!aligned16(qc) || !aligned16(kc)) return fail(BSA_ERR_INVALID_ARG, "centroids must be 16-byte aligned");
+  bsa::SelectArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.qc = qc; a.kc = kc; a.idx = idx; a.cnt = cnt; a.scores = scores; a.kmax = kmax;
+  a.mode = (int)mode;
+  a.scale = (float)(1.0 / std::sqrt((double)p->g.D));
+  for (int h = 0; h < p->g.Hd; ++h)
+    a.param[h] = mode == BSA_TOPK ? (double)k_for_density(param[h], p->g.nb) : param[h];
+  cudaError_t e = bsa::launch_select(p->g, a, st);
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "select kernel");
+}
+
+bsa_status run_attention(const bsa_plan_s* p, const void* q, const void* k, const void* v,
+                         const int32_t* idx, const int32_t* cnt, int kmax, void* o,
+                         int32_t* dev_status, cudaStream_t st) {
+  if (!q || !k || !v || !o) return fail(BSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(BSA_ERR_INVALID_ARG, "blocked tensors must be 16-byte aligned");
+  if (p->g.nb > 0 && (!idx || !cnt)) return fail(BSA_ERR_INVALID_ARG, "NULL index list");
+  if (kmax < 1) return fail(BSA_ERR_INVALID_ARG, "kmax must be >= 1");
+  bsa::AttnArgs a;
+  a.q = q; a.k = k; a.v = v; a.o = o; a.idx = idx; a.cnt = cnt; a.masks = p->d_masks;
+  a.status = dev_status ? dev_status : p->d_status;
+  a.kmax = kmax;
+  a.scale = (float)(1.0 / std::sqrt((double)p->g.D));
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->g.D));
+  cudaError_t e;
+  if (p->attn_path == 1) {
+    CUtensorMap tq, tk, tv;
+    const long long rows = (long long)p->g.B * p->g.Hd * p->g.npad_tot;
+    bsa_status s;
+    if ((s = make_tile_map(&tq, q, rows, p->g.D)) != BSA_OK) return s;
+    if ((s = make_tile_map(&tk, k, rows, p->g.D)) != BSA_OK) return s;
+    if ((s = make_tile_map(&tv, v, rows, p->g.D)) != BSA_OK) return s;
+    e = bsa::launch_attn_tc(p->g, a, tq, tk, tv, st);
+  } else {
+    e = bsa::launch_attn_simt(p->g, p->dtype == BSA_BF16, a, st);
+  }
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "attention kernel");
+}
+
+}  // namespace
+
+extern "C" {
+
+int bsa_version(void) { return BSA_VERSION; }
+
+const char* bsa_last_error_string(void) { return g_err.c_str(); }
+
+bsa_status bsa_plan_create(bsa_plan_t* out, int batch, int T, int H, int W, int bf, int br, int bc,
+                           int heads, int head_dim, int n_text, bsa_dtype dtype) {
+  if (out == nullptr) return fail(BSA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (batch < 1 || T < 1 || H < 1 || W < 1)
+    return fail(BSA_ERR_INVALID_ARG, "batch and grid extents must be >= 1");
+  if (bf < 1 || br < 1 || bc < 1) return fail(BSA_ERR_INVALID_ARG, "block extents must be >= 1");
+  if (heads < 1 || heads > BSA_MAX_HEADS)
+    return fail(BSA_ERR_INVALID_ARG, "heads must be in [1, %d]", BSA_MAX_HEADS);
+  if (head_dim != 64 && head_dim != 128) return fail(BSA_ERR_INVALID_ARG, "head_dim must be 64 or 128");
+  if (n_text < 0) return fail(BSA_ERR_INVALID_ARG, "n_text must be >= 0");
+  if (dtype != BSA_F32 && dtype != BSA_BF16) return fail(BSA_ERR_INVALID_ARG, "bad dtype");
+  const long long bs = (long long)bf * br * bc;
+  if (bs > 256) return fail(BSA_ERR_INVALID_ARG, "block size bf*br*bc = %lld exceeds 256", bs);
+
+  bsa_plan_s p;
+  Geo& g = p.g;
+  g.B = batch; g.T = T; g.H = H; g.W = W; g.bf = bf; g.br = br; g.bc = bc;
+  g.Hd = heads; g.D = head_dim; g.n_text = n_text;
+  g.nbt = (T + bf - 1) / bf; g.nby = (H + br - 1) / br; g.nbx = (W + bc - 1) / bc;
+  const long long nb = (long long)g.nbt * g.nby * g.nbx;
+  g.bs = (int)bs;
+  g.nb_text = (int)((n_text + bs - 1) / bs);
+  g.n_video = (long long)T * H * W;
+  g.n_tot = g.n_video + n_text;
+  const long long npad = (nb + g.nb_text) * bs;
+  g.npad_tot = npad;
+  if (nb > (1 << 24)) return fail(BSA_ERR_INVALID_ARG, "too many blocks");
+  g.nb = (int)nb;
+  if ((long long)batch * heads * npad >= (1ll << 31) || (long long)batch * g.n_tot * heads >= (1ll << 31))
+    return fail(BSA_ERR_UNSUPPORTED, "problem exceeds 2^31 rows");
+  if (bsa::select_smem_bytes(g.nb, head_dim) > 227 * 1024)
+    return fail(BSA_ERR_UNSUPPORTED, "nb = %d video blocks exceeds the selection kernel's limit", g.nb);
+  p.dtype = dtype;
+  p.attn_path = (dtype == BSA_BF16 && bs == 128) ? 1 : 0;
+  p.d_status = nullptr;
+  p.d_masks = nullptr;
+
+  cudaError_t e = cudaGetDevice(&p.device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  const int nbk = g.nb + g.nb_text;
+  std::vector<uint32_t> masks((size_t)nbk * 4, 0u);
+  if (bs <= 128)
+    for (int j = 0; j < nbk; ++j)
+      for (int s = 0; s < (int)bs; ++s)
+        if (slot_token(g, j, s) >= 0) masks[(size_t)j * 4 + s / 32] |= 1u << (s % 32);
+  e = cudaMalloc(&p.d_status, sizeof(int32_t));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(status)");
+  e = cudaMalloc(&p.d_masks, masks.size() * sizeof(uint32_t));
+  if (e != cudaSuccess) { cudaFree(p.d_status); return cuda_fail(e, "cudaMalloc(masks)"); }
+  if ((e = cudaMemset(p.d_status, 0, sizeof(int32_t))) != cudaSuccess ||
+      (e = cudaMemcpy(p.d_masks, masks.data(), masks.size() * sizeof(uint32_t),
+                      cudaMemcpyHostToDevice)) != cudaSuccess) {
+    cudaFree(p.d_status);
+    cudaFree(p.d_masks);
+    return cuda_fail(e, "plan upload");
+  }
+  *out = new bsa_plan_s(p);
+  return BSA_OK;
+}
+
+bsa_status bsa_plan_destroy(bsa_plan_t plan) {
+  if (plan == nullptr) return BSA_OK;
+  cudaFree(plan->d_status);
+  cudaFree(plan->d_masks);
+  delete plan;
+  return BSA_OK;
+}
+
+bsa_status bsa_plan_get_info(bsa_plan_t p, bsa_plan_info_t* info) {
+  if (p == nullptr || info == nullptr) return fail(BSA_ERR_INVALID_ARG, "NULL argument");
+  const Geo& g = p->g;
+  info->batch = g.B; info->T = g.T; info->H = g.H; info->W = g.W;
+  info->bf = g.bf; info->br = g.br; info->bc = g.bc; info->heads = g.Hd; info->head_dim = g.D;
+  info->n_text = g.n_text; info->dtype = (int)p->dtype;
+  info->Tp = g.nbt * g.bf; info->Hp = g.nby * g.br; info->Wp = g.nbx * g.bc;
+  info->nbt = g.nbt; info->nby = g.nby; info->nbx = g.nbx; info->nb = g.nb;
+  info->nb_text = g.nb_text; info->bs = g.bs;
+  info->n_video = g.n_video; info->n_tot = g.n_tot; info->npad_tot = g.npad_tot;
+  info->attn_path = p->attn_path;
+  return BSA_OK;
+}
+
+bsa_status bsa_kmax_for(bsa_plan_t p, bsa_select_mode mode, const double* param, int* kmax) {
+  if (p == nullptr || kmax == nullptr) return fail(BSA_ERR_INVALID_ARG, "NULL argument");
+  return check_params(p, mode, param, kmax);
+}
+
+bsa_status bsa_workspace_size(bsa_plan_t p, int kmax, size_t* select_ws, size_t* forward_ws) {
+  if (p == nullptr) return fail(BSA_ERR_INVALID_ARG, "plan is NULL");
+  if (kmax < 1) return fail(BSA_ERR_INVALID_ARG, "kmax must be >= 1");
+  const size_t cent = round256(cent_bytes(p));
+  const size_t lists = round256((size_t)p->g.B * p->g.Hd * p->g.nb * kmax * sizeof(int32_t)) +
+                       round256((size_t)p->g.B * p->g.Hd * p->g.nb * sizeof(int32_t));
+  if (select_ws) *select_ws = 2 * cent;
+  if (forward_ws) *forward_ws = 4 * round256(blk_bytes(p)) + 2 * cent + lists;
+  return BSA_OK;
+}
+
+bsa_status bsa_permute(bsa_plan_t p, const void* x, void* x_blk, float* centroids, void* stream) {
+  bsa_status s = check_plan(p);
+  if (s != BSA_OK) return s;
+  if (!x || !x_blk) return fail(BSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(x) || !aligned16(x_blk) || (centroids && !aligned16(centroids)))
+    return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  bsa::GatherArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.src[0] = x; a.dst[0] = x_blk; a.cent[0] = centroids; a.ntensors = 1;
+  cudaError_t e = bsa::launch_permute(p->g, p->dtype == BSA_BF16, a, (cudaStream_t)stream);
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "permute kernel");
+}
+
+bsa_status bsa_permute_qkv(bsa_plan_t p, const void* q, const void* k, const void* v, void* q_blk,
+                           void* k_blk, void* v_blk, float* q_cent, float* k_cent, void* stream) {
+  bsa_status s = check_plan(p);
+  if (s != BSA_OK) return s;
+  if (!q || !k || !v || !q_blk || !k_blk || !v_blk) return fail(BSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  const void* ptrs[8] = {q, k, v, q_blk, k_blk, v_blk, q_cent, k_cent};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  bsa::GatherArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.src[0] = q; a.src[1] = k; a.src[2] = v;
+  a.dst[0] = q_blk; a.dst[1] = k_blk; a.dst[2] = v_blk;
+  a.cent[0] = q_cent; a.cent[1] = k_cent; a.cent[2] = nullptr;
+  a.ntensors = 3;
+  cudaError_t e = bsa::launch_permute(p->g, p->dtype == BSA_BF16, a, (cudaStream_t)stream);
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "permute kernel");
+}
+
+bsa_status bsa_unpermute(bsa_plan_t p, const void* o_blk, void* o, void* stream) {
+  bsa_status s = check_plan(p);
+  if (s != BSA_OK) return s;
+  if (!o_blk || !o) return fail(BSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(o_blk) || !aligned16(o)) return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  bsa::GatherArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.src[0] = o_blk; a.dst[0] = o; a.ntensors = 1;
+  cudaError_t e = bsa::launch_unpermute(p->g, p->dtype == BSA_BF16, a, (cudaStream_t)stream);
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "unpermute kernel");
+}
+
+bsa_status bsa_select(bsa_plan_t p, const void* q_blk, const void* k_blk, bsa_select_mode mode,
+                      const double* param, int kmax, int32_t* idx, int32_t* cnt, float* scores,
+                      void* ws, size_t ws_bytes, void* stream) {
+  bsa_status s = check_plan(p);
+  if (s != BSA_OK) return s;
+  int need = 0;
+  if ((s = check_params(p, mode, param, &need)) != BSA_OK) return s;
+  if (kmax < need) return fail(BSA_ERR_INVALID_ARG, "kmax %d is below the %d entries a list can need", kmax, need);
+  if (!q_blk || !k_blk) return fail(BSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q_blk) || !aligned16(k_blk)) return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  size_t need_ws = 0;
+  bsa_workspace_size(p, kmax, &need_ws, nullptr);
+  if (ws == nullptr || ws_bytes < need_ws)
+    return fail(BSA_ERR_WORKSPACE, "select needs %zu bytes of workspace, got %zu", need_ws, ws_bytes);
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(BSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  float* qc = reinterpret_cast<float*>(ws);
+  float* kc = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + round256(cent_bytes(p)));
+  bsa::GatherArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.src[0] = q_blk; a.src[1] = k_blk; a.cent[0] = qc; a.cent[1] = kc; a.ntensors = 2;
+  cudaError_t e = bsa::launch_pool(p->g, p->dtype == BSA_BF16, a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "centroid kernel");
+  return run_select(p, qc, kc, mode, param, kmax, idx, cnt, scores, (cudaStream_t)stream);
+}
+
+bsa_status bsa_select_centroids(bsa_plan_t p, const float* q_cent, const float* k_cent,
+                                bsa_select_mode mode, const double* param, int kmax, int32_t* idx,
+                                int32_t* cnt, float* scores, void* stream) {
+  bsa_status s = check_plan(p);
+  if (s != BSA_OK) return s;
+  return run_select(p, q_cent, k_cent, mode, param, kmax, idx, cnt, scores, (cudaStream_t)stream);
+}
+
+bsa_status bsa_attention(bsa_plan_t p, const void* q_blk, const void* k_blk, const void* v_blk,
+                         const int32_t* idx, const int32_t* cnt, int kmax, void* o_blk,
+                         int32_t* dev_status, void* stream) {
+  bsa_status s = check_plan(p);
+  if (s != BSA_OK) return s;
+  return run_attention(p, q_blk, k_blk, v_blk, idx, cnt, kmax, o_blk, dev_status, (cudaStream_t)stream);
+}
+
+bsa_status bsa_forward(bsa_plan_t p, const void* q, const void* k, const void* v,
+                       bsa_select_mode mode, const double* param, int kmax, void* o,
+                       int32_t* idx_out, int32_t* cnt_out, void* ws, size_t ws_bytes,
+                       int32_t* dev_status, void* stream) {
+  bsa_status s = check_plan(p);
+  if (s != BSA_OK) return s;
+  int need = 0;
+  if ((s = check_params(p, mode, param, &need)) != BSA_OK) return s;
+  if (kmax < need) return fail(BSA_ERR_INVALID_ARG, "kmax %d is below the %d entries a list can need", kmax, need);
+  if (!q || !k || !v || !o) return fail(BSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  size_t need_ws = 0;
+  bsa_workspace_size(p, kmax, nullptr, &need_ws);
+  if (ws == nullptr || ws_bytes < need_ws)
+    return fail(BSA_ERR_WORKSPACE, "forward needs %zu bytes of workspace, got %zu", need_ws, ws_bytes);
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(BSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  char* w = reinterpret_cast<char*>(ws);
+  const size_t tb = round256(blk_bytes(p)), cb = round256(cent_bytes(p));
+  void* q_blk = w; w += tb;
+  void* k_blk = w; w += tb;
+  void* v_blk = w; w += tb;
+  void* o_blk = w; w += tb;
+  float* qc = reinterpret_cast<float*>(w); w += cb;
+  float* kc = reinterpret_cast<float*>(w); w += cb;
+  int32_t* idx = reinterpret_cast<int32_t*>(w);
+  w += round256((size_t)p->g.B * p->g.Hd * p->g.nb * kmax * sizeof(int32_t));
+  int32_t* cnt = reinterpret_cast<int32_t*>(w);
+  if (idx_out) idx = idx_out;
+  if (cnt_out) cnt = cnt_out;
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((s = bsa_permute_qkv(p, q, k, v, q_blk, k_blk, v_blk, qc, kc, stream)) != BSA_OK) return s;
+  if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st)) != BSA_OK) return s;
+  if ((s = run_attention(p, q_blk, k_blk, v_blk, idx, cnt, kmax, o_blk, dev_status, st)) != BSA_OK) return s;
+  return bsa_unpermute(p, o_blk, o, stream);
+}
+
+bsa_status bsa_check_status(bsa_plan_t p, void* stream) {
+  bsa_status s = check_plan(p);
+  if (s != BSA_OK) return s;
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int32_t v = 0;
+  if ((e = cudaMemcpy(&v, p->d_status, sizeof(v), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "status read");
+  if ((e = cudaMemset(p->d_status, 0, sizeof(v))) != cudaSuccess) return cuda_fail(e, "status reset");
+  if (v == 0) return BSA_OK;
+  return fail((bsa_status)v, "kernel reported status %d (%s)", v,
+              v == BSA_ERR_TIMEOUT ? "a bounded wait ran out" : "an index list entry was out of range");
+}
+
+}  // extern "C"

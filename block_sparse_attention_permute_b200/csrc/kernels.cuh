@@ -1,0 +1,54 @@
+// kernels.cuh — argument blocks and launchers of the libbsa kernels
+// (internal; the public interface is include/bsa.h).
+#pragma once
+#include "common.cuh"
+
+namespace bsa {
+
+struct GatherArgs {
+  const void* src[3];
+  void* dst[3];      // unused in kPool
+  float* cent[3];    // optional centroid outputs (kPermute, kPool)
+  int ntensors;
+};
+
+struct SelectArgs {
+  const float* qc;   // [B, Hd, nb, D]
+  const float* kc;   // [B, Hd, nb, D]
+  int32_t* idx;      // [B, Hd, nb, kmax]
+  int32_t* cnt;      // [B, Hd, nb]
+  float* scores;     // [B, Hd, nb, nb] or null
+  int kmax;
+  int mode;          // 0 top-k, 1 top-p
+  float scale;       // 1/sqrt(D) rounded to fp32
+  double param[BSA_MAX_HEADS];  // k (held in a double) or tau, per head
+};
+
+struct AttnArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  const int32_t* idx;     // [B, Hd, nb, kmax]
+  const int32_t* cnt;     // [B, Hd, nb]
+  const uint32_t* masks;  // [(nb + nb_text) * 4] slot validity bits (bs == 128 only)
+  int32_t* status;        // device status word
+  int kmax;
+  float scale;            // 1/sqrt(D)
+  float scale_log2;       // log2(e)/sqrt(D)
+};
+
+// permute.cu
+cudaError_t launch_permute(const Geo& g, bool is_bf16, const GatherArgs& a, cudaStream_t st);
+cudaError_t launch_unpermute(const Geo& g, bool is_bf16, const GatherArgs& a, cudaStream_t st);
+cudaError_t launch_pool(const Geo& g, bool is_bf16, const GatherArgs& a, cudaStream_t st);
+// select.cu
+size_t select_smem_bytes(int nb, int D);
+cudaError_t launch_select(const Geo& g, const SelectArgs& a, cudaStream_t st);
+// attn.cu
+size_t attn_tc_smem_bytes(int D);
+cudaError_t launch_attn_simt(const Geo& g, bool is_bf16, const AttnArgs& a, cudaStream_t st);
+cudaError_t launch_attn_tc(const Geo& g, const AttnArgs& a, const CUtensorMap& tq,
+                           const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st);
+
+}  // namespace bsa

@@ -1,0 +1,205 @@
+// select.cu — index search: centroid score matrix + head-wise Top-K / Top-P.
+//
+// SPADE (arXiv 2608.03335) §3.3: "From Q'/K' we compute ... an inter-block
+// importance matrix of size N_Qblocks x N_Kblocks via the inter-estimator.
+// Scores are filtered by Top-K or Top-P."  §3.1: MEAN-SPADE estimates with
+// (q_mean, k_mean); "the dot product of blue vectors gives inter-block
+// importance"; Top-K keep or Top-P cumulative threshold per head.
+//
+// Scores: s_ij = qbar_i . kbar_j * (1/sqrt(D)) in fp32 (one fma chain over d
+// in ascending order, so the value does not depend on the launch shape);
+// p_ij = e_ij / Z_i with e_ij = expf(s_ij - max_j s_ij) and Z_i summed in fp64.
+// Selection, one warp per query-block row:
+//   Top-K: the k-th largest score is found by a 32-step bitwise search over
+//          the order-preserving integer image of s; equal scores are taken in
+//          ascending block id.
+//   Top-P: the largest score threshold whose mass sum_{s_j >= t} e_j reaches
+//          tau * Z (fp64), then ties at the threshold in ascending block id
+//          until the mass is reached: the shortest prefix in descending order.
+// Lists are written in ascending block id; the text key blocks follow.
+#include "kernels.cuh"
+
+namespace bsa {
+
+
+constexpr int kSelRows = 16;      // query-block rows per CTA
+constexpr int kSelKeys = 64;      // key blocks per score chunk
+constexpr int kSelThreads = 256;  // 8 warps
+
+size_t select_smem_bytes(int nb, int D) {
+  return sizeof(float) *
+         ((size_t)kSelRows * D + (size_t)kSelKeys * (D + 4) + (size_t)kSelRows * nb);
+}
+
+__device__ __forceinline__ uint32_t order_key(float s) {
+  const uint32_t u = __float_as_uint(s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Sum over the warp, the same value in every lane (tree to lane 0, broadcast).
+__device__ __forceinline__ double warp_sum_uniform(double v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_down_sync(0xffffffffu, v, off);
+  return __shfl_sync(0xffffffffu, v, 0);
+}
+
+__device__ __forceinline__ int warp_count(bool pred) {
+  return __popc(__ballot_sync(0xffffffffu, pred));
+}
+
+// sum over j with key(s_j) >= cand of expf(s_j - m), in fp64, fixed order.
+__device__ double mass_at_least(const float* row, int nb, float m, uint32_t cand, int lane) {
+  double acc = 0.0;
+  for (int j = lane; j < nb; j += 32) {
+    const float s = row[j];
+    if (order_key(s) >= cand) acc += (double)expf(s - m);
+  }
+  return warp_sum_uniform(acc);
+}
+
+__device__ int count_at_least(const float* row, int nb, uint32_t cand, int lane) {
+  int c = 0;
+  for (int j = lane; j < nb; j += 32) c += order_key(row[j]) >= cand ? 1 : 0;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+  return c;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, SelectArgs a) {
+  extern __shared__ __align__(16) float sm[];
+  float* qs = sm;                                   // [kSelRows][D]
+  float* ks = qs + kSelRows * D;                    // [kSelKeys][D+4]
+  float* sc = ks + kSelKeys * (D + 4);              // [kSelRows][nb]
+  const int nb = g.nb;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const long long bh = (long long)b * g.Hd + h;
+  const int i0 = blockIdx.x * kSelRows;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  // ---- phase 1: scores of kSelRows query blocks against all key blocks ----
+  for (int e = tid; e < kSelRows * D; e += kSelThreads) {
+    const int r = e / D, d = e % D;
+    qs[e] = (i0 + r < nb) ? a.qc[(bh * nb + i0 + r) * D + d] : 0.f;
+  }
+  const int tx = tid % kSelKeys;     // key within chunk
+  const int ty = tid / kSelKeys;     // row group: rows 4*ty .. 4*ty+3
+  for (int j0 = 0; j0 < nb; j0 += kSelKeys) {
+    __syncthreads();
+    for (int e = tid; e < kSelKeys * (D / 4); e += kSelThreads) {
+      const int jj = e / (D / 4), d4 = e % (D / 4);
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j0 + jj < nb) v = *reinterpret_cast<const float4*>(a.kc + (bh * nb + j0 + jj) * D + 4 * d4);
+      *reinterpret_cast<float4*>(ks + jj * (D + 4) + 4 * d4) = v;
+    }
+    __syncthreads();
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int d4 = 0; d4 < D / 4; ++d4) {
+      const float4 kv = *reinterpret_cast<const float4*>(ks + tx * (D + 4) + 4 * d4);
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        const float4 qv = *reinterpret_cast<const float4*>(qs + (4 * ty + rr) * D + 4 * d4);
+        acc[rr] = fmaf(qv.x, kv.x, acc[rr]);
+        acc[rr] = fmaf(qv.y, kv.y, acc[rr]);
+        acc[rr] = fmaf(qv.z, kv.z, acc[rr]);
+        acc[rr] = fmaf(qv.w, kv.w, acc[rr]);
+      }
+    }
+    if (j0 + tx < nb) {
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) sc[(4 * ty + rr) * nb + j0 + tx] = acc[rr] * a.scale + 0.0f;
+    }
+  }
+  __syncthreads();
+
+  // ---- phase 2: one warp per row: softmax statistics and selection ----
+  for (int r = warp; r < kSelRows; r += kSelThreads / 32) {
+    const int i = i0 + r;
+    if (i >= nb) break;
+    const float* row = sc + r * nb;
+    float m = -INFINITY;
+    for (int j = lane; j < nb; j += 32) m = fmaxf(m, row[j]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const double Z = mass_at_least(row, nb, m, 0u, lane);
+
+    if (a.scores != nullptr) {
+      float* out = a.scores + (bh * nb + i) * nb;
+      for (int j = lane; j < nb; j += 32) out[j] = (float)((double)expf(row[j] - m) / Z);
+    }
+
+    uint32_t T = 0;
+    int need = 0;  // how many of the scores equal to the threshold to take
+    if (a.mode == 0) {
+      const int k = (int)a.param[h];
+      for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = T | (1u << bit);
+        if (count_at_least(row, nb, cand, lane) >= k) T = cand;
+      }
+      const int n_gt = (T == 0xffffffffu) ? 0 : count_at_least(row, nb, T + 1, lane);
+      need = k - n_gt;
+    } else {
+      const double target = a.param[h] * Z;
+      for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = T | (1u << bit);
+        if (mass_at_least(row, nb, m, cand, lane) >= target) T = cand;
+      }
+      double acc = (T == 0xffffffffu) ? 0.0 : mass_at_least(row, nb, m, T + 1, lane);
+      int n_eq = 0;
+      float s_eq = 0.f;
+      for (int j = lane; j < nb; j += 32)
+        if (order_key(row[j]) == T) { ++n_eq; s_eq = row[j]; }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        n_eq += __shfl_xor_sync(0xffffffffu, n_eq, off);
+        s_eq = fmaxf(s_eq, __shfl_xor_sync(0xffffffffu, s_eq, off));
+      }
+      const double e_eq = (double)expf(s_eq - m);
+      while (acc < target && need < n_eq) {
+        acc += e_eq;
+        ++need;
+      }
+      if (need == 0) need = 1;
+    }
+
+    // Ascending compaction of {key > T} plus the first `need` of {key == T}.
+    int32_t* out = a.idx + (bh * nb + i) * a.kmax;
+    int written = 0, eq_seen = 0;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (int j0 = 0; j0 < nb; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t key = j < nb ? order_key(row[j]) : 0u;
+      const bool gt = j < nb && key > T;
+      const bool eq = j < nb && key == T;
+      const uint32_t eq_bal = __ballot_sync(0xffffffffu, eq);
+      const bool take = gt || (eq && eq_seen + __popc(eq_bal & lt_mask) < need);
+      const uint32_t sel_bal = __ballot_sync(0xffffffffu, take);
+      if (take) out[written + __popc(sel_bal & lt_mask)] = j;
+      written += __popc(sel_bal);
+      eq_seen += __popc(eq_bal);
+    }
+    for (int t = lane; t < g.nb_text; t += 32) out[written + t] = nb + t;
+    if (lane == 0) a.cnt[bh * nb + i] = written + g.nb_text;
+  }
+}
+
+cudaError_t launch_select(const Geo& g, const SelectArgs& a, cudaStream_t st) {
+  const size_t smem = select_smem_bytes(g.nb, g.D);
+  dim3 grid((g.nb + kSelRows - 1) / kSelRows, g.Hd, g.B);
+  cudaError_t e;
+  if (g.D == 128) {
+    e = cudaFuncSetAttribute(select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    select_kernel<128><<<grid, kSelThreads, smem, st>>>(g, a);
+  } else {
+    e = cudaFuncSetAttribute(select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    select_kernel<64><<<grid, kSelThreads, smem, st>>>(g, a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace bsa

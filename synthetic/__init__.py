@@ -17,8 +17,9 @@ trained weights; the shapes are those models' latent grids):
     0.3 * N(0, 1).
   * bf16 workloads: Q and K (text included) are multiplied by a common
     per-head factor s so that the standard deviation of q.k/sqrt(D) over 4096
-    seeded random (video query, video key) pairs is 3; V is not scaled.  The
-    result is rounded to bf16 (round to nearest even).
+    seeded random (video query, video key) pairs is 3 (factor 1 when those
+    pairs have no spread, e.g. a one-token grid); V is not scaled.  The result
+    is rounded to bf16 (round to nearest even).
   * Per-head mixed density (Wan2.1-14B shape): u ~ U[0, 1) per head (seed 4);
     rho = 0.03 if u < 0.35, 0.05 if u < 0.50, else 0.10.
 """
@@ -169,7 +170,9 @@ def make_custom(B, T, H, W, Hd, D, n_text=0, dtype="bf16", qk_std=3.0, seed_base
         for b in range(B):
             for h in range(Hd):
                 dots = (q[b, qi, h, :].double() * k[b, ki, h, :].double()).sum(-1) / math.sqrt(D)
-                s = math.sqrt(qk_std / float(dots.std()))
+                sd = float(dots.std())
+                # a grid of one token (every sampled pair is the same pair) has no spread
+                s = math.sqrt(qk_std / sd) if sd > 1e-3 else 1.0
                 q[b, :, h, :] *= s
                 k[b, :, h, :] *= s
     dt = torch.float32 if dtype == "f32" else torch.bfloat16

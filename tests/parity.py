@@ -1,0 +1,103 @@
+"""Shared helpers of the GPU parity tests: CUDA path vs the fp64 oracle.
+
+Tolerances (from the stated bar):
+  * layouts, index lists and counts: bit-exact, except rows the oracle
+    reports as ties (k-th and (k+1)-th scores, or the Top-P cumulative mass
+    at the cut, within 1e-5 relative); such rows must still be a valid
+    selection within that tolerance.
+  * attention output, bf16 inputs: max-abs <= 2e-2 and mean-abs <= 2e-3.
+  * attention output, fp32 inputs: max-abs <= 1e-5.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle as orc
+import synthetic
+
+TOL_BF16_MAX, TOL_BF16_MEAN = 2e-2, 2e-3
+TOL_F32_MAX = 1e-5
+TIE_REL = 1e-5
+
+
+def geometry(w) -> orc.Geometry:
+    return orc.Geometry(*w.geometry_args())
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy() if t.dtype == torch.bfloat16 else t.detach().cpu().numpy()
+
+
+def check_lists(g, gpu_idx, gpu_cnt, o_idx, o_cnt, tie, p, mode, params):
+    """Bit-exact lists on non-tie rows; valid selections on tie rows. Returns #ties."""
+    gi, gc = gpu_idx.cpu().numpy(), gpu_cnt.cpu().numpy()
+    assert gc.shape == o_cnt.shape
+    n_tie = 0
+    for b in range(g.B):
+        for h in range(g.Hd):
+            for i in range(g.nb):
+                c = int(gc[b, h, i])
+                lst = list(gi[b, h, i, :c])
+                ref = list(o_idx[b, h, i, :o_cnt[b, h, i]])
+                if lst == ref:
+                    continue
+                assert tie[b, h, i], f"list mismatch at b={b} h={h} i={i}: {lst[:8]}... vs {ref[:8]}..."
+                n_tie += 1
+                text = list(range(g.nb, g.nb + g.nb_text))
+                assert lst[len(lst) - g.nb_text:] == text
+                sel = np.array(lst[:len(lst) - g.nb_text], dtype=np.int64)
+                assert np.all(np.diff(sel) > 0) and sel.min() >= 0 and sel.max() < g.nb
+                row = p[b, h, i]
+                uns = np.setdiff1d(np.arange(g.nb), sel)
+                if len(uns):
+                    assert row[sel].min() >= row[uns].max() * (1 - TIE_REL) - 1e-300
+                if mode == 0:
+                    assert len(sel) == orc.k_for_density(params[h], g.nb)
+                else:
+                    tau = params[h]
+                    mass = row[sel].sum()
+                    assert mass >= tau * (1 - TIE_REL)
+                    assert mass - row[sel].min() < tau * (1 + TIE_REL)
+    return n_tie
+
+
+def check_output(gpu, ref, dtype_name, what=""):
+    """Elementwise comparison at the stated tolerance; returns (max_abs, mean_abs)."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    assert np.all(np.isfinite(gpu)), f"{what}: non-finite output"
+    err = np.abs(gpu - ref)
+    mx, mean = float(err.max()), float(err.mean())
+    if dtype_name == "f32":
+        assert mx <= TOL_F32_MAX, f"{what}: max-abs {mx:.3e} > {TOL_F32_MAX}"
+    else:
+        assert mx <= TOL_BF16_MAX, f"{what}: max-abs {mx:.3e} > {TOL_BF16_MAX}"
+        assert mean <= TOL_BF16_MEAN, f"{what}: mean-abs {mean:.3e} > {TOL_BF16_MEAN}"
+    return mx, mean
+
+
+def sample_rows(g, seed=0, n_blocks=6, n_text=16):
+    """Token rows for sampled comparison: all valid tokens of a few random video
+    blocks, always the last (most padded) block, plus some text tokens."""
+    rng = np.random.default_rng(seed)
+    blocks = set(rng.choice(g.nb, size=min(n_blocks, g.nb), replace=False).tolist())
+    blocks.add(g.nb - 1)
+    rows = []
+    for j in sorted(blocks):
+        tb, yb, xb = j // (g.nby * g.nbx), (j // g.nbx) % g.nby, j % g.nbx
+        for t in range(tb * g.bf, min(g.T, (tb + 1) * g.bf)):
+            for y in range(yb * g.br, min(g.H, (yb + 1) * g.br)):
+                for x in range(xb * g.bc, min(g.W, (xb + 1) * g.bc)):
+                    rows.append((t * g.H + y) * g.W + x)
+    if g.n_text:
+        rows += sorted(rng.choice(g.n_text, size=min(n_text, g.n_text), replace=False)
+                       + g.n_video)
+    return np.array(rows, dtype=np.int64)
+
+
+def custom_workload(name, B, T, H, W, bf, br, bc, Hd, D, n_text, dtype, mode, param):
+    w = synthetic.Workload(name, B, T, H, W, bf, br, bc, Hd, D, dtype, mode, [param] * Hd,
+                           n_text=n_text, qk_std=3.0 if dtype == "bf16" else None)
+    return w

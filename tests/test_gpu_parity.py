@@ -1,0 +1,172 @@
+"""GPU parity: every step of the CUDA path (through the C ABI) against the fp64
+oracle on the same seeded inputs.
+
+Small cases (several tiles, ragged tails, text blocks, both head dims, both
+selection modes, both attention kernels) are compared element by element.
+The full workloads are compared in the launch configuration bench.py times
+(bsa_forward): index lists in full, outputs on sampled rows.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_permute_b200 as bsa
+import oracle as orc
+import synthetic
+from parity import (check_lists, check_output, custom_workload, geometry, sample_rows, to_np)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny": synthetic.workload("tiny"),
+    "hy_ragged_text": custom_workload("hy_ragged_text", 1, 6, 12, 20, 1, 8, 16, 3, 128, 130,
+                                      "bf16", 0, 0.3),
+    "wan_d64_b2": custom_workload("wan_d64_b2", 2, 9, 10, 20, 4, 4, 8, 2, 64, 0, "bf16", 0, 0.25),
+    "wan_topp": custom_workload("wan_topp", 1, 9, 10, 20, 4, 4, 8, 3, 128, 0, "bf16", 1, 0.9),
+    "simt_bf16_bs32": custom_workload("simt_bf16_bs32", 1, 5, 9, 12, 2, 4, 4, 2, 128, 40, "bf16",
+                                      0, 0.3),
+    "f32_bs128": custom_workload("f32_bs128", 1, 6, 12, 20, 1, 8, 16, 2, 64, 0, "f32", 0, 0.3),
+    "dense_rho1": custom_workload("dense_rho1", 1, 4, 16, 16, 1, 8, 16, 2, 128, 0, "bf16", 0, 1.0),
+    "k_is_one": custom_workload("k_is_one", 1, 8, 16, 16, 2, 4, 16, 2, 128, 0, "bf16", 0, 0.001),
+    "topp_tau1": custom_workload("topp_tau1", 1, 8, 16, 16, 2, 4, 16, 2, 128, 0, "bf16", 1, 1.0),
+    "single_token": custom_workload("single_token", 1, 1, 1, 1, 1, 8, 16, 1, 128, 0, "bf16", 0, 1.0),
+}
+
+
+@pytest.fixture(scope="module")
+def dev():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    bsa.load()
+    return torch.device("cuda", 0)
+
+
+def _inputs(w, dev):
+    q, k, v = synthetic.make_qkv(w)
+    return (q, k, v), (q.to(dev), k.to(dev), v.to(dev))
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_permute_and_centroids(name, dev):
+    w = SMALL[name]
+    g = geometry(w)
+    (q, _, _), (qd, _, _) = _inputs(w, dev)
+    plan = bsa.plan_for(w, dev)
+    qb, qc = plan.permute(qd, centroids=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(qb).astype(np.float64), orc.permute(g, to_np(q)))
+    ref_c = orc.centroids(g, to_np(q))
+    np.testing.assert_allclose(qc.cpu().numpy(), ref_c, rtol=1e-5, atol=1e-5)
+    back = plan.unpermute(qb)
+    torch.cuda.synchronize()
+    assert torch.equal(back.cpu(), q)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_select_lists_and_scores(name, dev):
+    w = SMALL[name]
+    g = geometry(w)
+    (q, k, _), (qd, kd, _) = _inputs(w, dev)
+    plan = bsa.plan_for(w, dev)
+    qb, qc = plan.permute(qd, centroids=True)
+    kb, kc = plan.permute(kd, centroids=True)
+    idx, cnt, sc = plan.select(qb, kb, w.mode, w.params, scores=True)
+    idx2, cnt2 = plan.select_centroids(qc, kc, w.mode, w.params)
+    torch.cuda.synchronize()
+    p = orc.scores(g, orc.centroids(g, to_np(q)), orc.centroids(g, to_np(k)))
+    o_idx, o_cnt, tie = orc.select(g, p, w.mode, w.params)
+    check_lists(g, idx, cnt, o_idx, o_cnt, tie, p, w.mode, w.params)
+    # the pooled and the fused-permute centroids give the same lists
+    assert torch.equal(cnt, cnt2)
+    for b, h, i in np.ndindex(*cnt.shape):
+        c = int(cnt[b, h, i])
+        assert torch.equal(idx[b, h, i, :c], idx2[b, h, i, :c])
+    np.testing.assert_allclose(sc.cpu().numpy(), p, rtol=2e-5, atol=1e-7)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_attention_and_forward(name, dev):
+    w = SMALL[name]
+    g = geometry(w)
+    (q, k, v), (qd, kd, vd) = _inputs(w, dev)
+    plan = bsa.plan_for(w, dev)
+    qb, kb, vb, qc, kc = plan.permute_qkv(qd, kd, vd)
+    idx, cnt = plan.select_centroids(qc, kc, w.mode, w.params)
+    ob = plan.attention(qb, kb, vb, idx, cnt)
+    out, fidx, fcnt = plan.forward(qd, kd, vd, w.mode, w.params, return_lists=True)
+    plan.check_status()
+    gi, gc = idx.cpu().numpy(), cnt.cpu().numpy()
+    ref = orc.attention(g, to_np(q), to_np(k), to_np(v), gi, gc)
+    check_output(to_np(ob), orc.permute(g, ref.astype(np.float32)), w.dtype, f"{name} blocked")
+    # pad rows of the blocked output are exactly zero
+    pad = np.ones(g.npad_tot, dtype=bool)
+    perm_ids = orc.permute(g, np.ones((g.B, g.n_tot, g.Hd, g.D), dtype=np.float32))[0, 0, :, 0]
+    pad[perm_ids == 1.0] = False
+    assert np.all(to_np(ob)[:, :, pad, :] == 0)
+    assert torch.equal(fcnt, cnt)
+    check_output(to_np(out), ref, w.dtype, f"{name} forward")
+
+
+def test_ones_values_give_ones(dev):
+    w = SMALL["hy_ragged_text"]
+    (_, _, _), (qd, kd, vd) = _inputs(w, dev)
+    plan = bsa.plan_for(w, dev)
+    out = plan.forward(qd, kd, torch.ones_like(vd), w.mode, w.params)
+    torch.cuda.synchronize()
+    assert torch.allclose(out.float(), torch.ones_like(out.float()), atol=1e-2, rtol=0)
+
+
+@pytest.mark.parametrize("path", ["hy_ragged_text", "simt_bf16_bs32"])
+def test_empty_and_bad_lists_are_handled(path, dev):
+    w = SMALL[path]
+    g = geometry(w)
+    (q, k, v), (qd, kd, vd) = _inputs(w, dev)
+    plan = bsa.plan_for(w, dev)
+    qb, kb, vb, qc, kc = plan.permute_qkv(qd, kd, vd)
+    idx, cnt = plan.select_centroids(qc, kc, w.mode, w.params)
+    # empty list on query block 0 -> its rows are zero; out-of-range entry on
+    # block 1 -> skipped and reported
+    cnt2, idx2 = cnt.clone(), idx.clone()
+    cnt2[0, 0, 0] = 0
+    idx2[0, 0, 1, 0] = g.nb + g.nb_text + 5
+    ob = plan.attention(qb, kb, vb, idx2, cnt2)
+    with pytest.raises(bsa.BsaError) as e:
+        plan.check_status()
+    assert e.value.status == 6
+    blk = to_np(ob)
+    assert np.all(blk[0, 0, :g.bs] == 0)
+    # block 1 equals attention over its list without the bad first entry
+    gi, gc = idx2.cpu().numpy().copy(), cnt2.cpu().numpy().copy()
+    c = gc[0, 0, 1]
+    gi[0, 0, 1, :c - 1] = gi[0, 0, 1, 1:c]
+    gc[0, 0, 1] = c - 1
+    ref = orc.permute(g, orc.attention(g, to_np(q), to_np(k), to_np(v), gi, gc).astype(np.float32))
+    check_output(blk[0, 0, g.bs:2 * g.bs], ref[0, 0, g.bs:2 * g.bs], w.dtype, "bad-index row")
+    plan.check_status()  # status was cleared
+
+
+# ------------------------------------------------------------ full workloads
+FULL = ["wan13", "hunyuan", "hunyuan20", "wan14", "wan14_topp", "long"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_workload_forward(name, dev):
+    w = synthetic.workload(name)
+    g = geometry(w)
+    (q, k, v), (qd, kd, vd) = _inputs(w, dev)
+    plan = bsa.plan_for(w, dev)
+    out, idx, cnt = plan.forward(qd, kd, vd, w.mode, w.params, return_lists=True)
+    plan.check_status()
+    qn, kn, vn = to_np(q), to_np(k), to_np(v)
+    p = orc.scores(g, orc.centroids(g, qn), orc.centroids(g, kn))
+    o_idx, o_cnt, tie = orc.select(g, p, w.mode, w.params)
+    n_tie = check_lists(g, idx, cnt, o_idx, o_cnt, tie, p, w.mode, w.params)
+    if w.mode == 0:
+        ks = np.array([orc.k_for_density(r, g.nb) for r in w.params])
+        assert np.all(cnt.cpu().numpy() == (ks[None, :, None] + g.nb_text))
+    rows = sample_rows(g, seed=zlib.crc32(name.encode()) % 1000)
+    ref = orc.attention(g, qn, kn, vn, idx.cpu().numpy(), cnt.cpu().numpy(), rows=rows)
+    got = out[:, torch.from_numpy(rows).to(dev)]
+    mx, mean = check_output(to_np(got), ref, w.dtype, name)
+    print(f"{name}: ties={n_tie} max_abs={mx:.3e} mean_abs={mean:.3e} rows={len(rows)}")
