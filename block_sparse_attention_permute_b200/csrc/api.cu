@@ -411,3 +411,15 @@ bsa_status bsa_check_status(bsa_plan_t p, void* stream) {
 }
 
 }  // extern "C"
+
+// Internal helpers for select_static.cu (C++ linkage, not part of the C ABI).
+bsa_status bsa_internal_fail(bsa_status s, const char* msg) { return fail(s, "%s", msg); }
+
+bsa_status bsa_internal_plan_sizes(bsa_plan_t p, const Geo** g, int* is_bf16, int* device) {
+  bsa_status s = check_plan(p);
+  if (s != BSA_OK) return s;
+  *g = &p->g;
+  *is_bf16 = p->dtype == BSA_BF16 ? 1 : 0;
+  *device = p->device;
+  return BSA_OK;
+}

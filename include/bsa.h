@@ -170,6 +170,28 @@ bsa_status bsa_select_centroids(bsa_plan_t plan, const float* q_cent,
                                 int32_t* idx, int32_t* cnt, float* scores,
                                 void* stream);
 
+/* bsa_select_static — bsa_select for callers that cannot allocate device
+ * memory.  The paper has no counterpart to this call; it exists for engines
+ * and plugin hosts that plan all device memory before serving and forbid
+ * allocation afterwards, and for hot loops that must not pay cudaMalloc's
+ * implicit synchronisation.  It takes no workspace and calls no allocator:
+ * the Q and K centroids live in a fixed 16 MiB device array inside libbsa,
+ * which every GPU that loads the library holds until the process exits.
+ *   Arguments, outputs and results are those of bsa_select.
+ *   Limit: 2 * batch * heads * nb * head_dim * 4 bytes (each half rounded up
+ *   to 256 bytes) must fit in 16 MiB, else BSA_ERR_UNSUPPORTED and nothing is
+ *   launched.
+ *   The first call on a device looks up that device's copy of the array
+ *   (cudaGetSymbolAddress, with the device current) and caches it; make that
+ *   first call before any stream capture begins.
+ *   All calls on a device share the array and it keeps the last call's
+ *   contents (each call rewrites every centroid it reads, so nothing needs
+ *   clearing); calls whose kernels overlap on the GPU race on it. */
+bsa_status bsa_select_static(bsa_plan_t plan, const void* q_blk, const void* k_blk,
+                             bsa_select_mode mode, const double* param_per_head,
+                             int kmax, int32_t* idx, int32_t* cnt, float* scores,
+                             void* stream);
+
 /* bsa_attention — flash block-sparse attention (SPADE §2.2 Eq. (2) with M = 0
  * on selected block pairs and valid keys, -inf elsewhere; §3.3 (3): online
  * softmax, no dense score matrix).
