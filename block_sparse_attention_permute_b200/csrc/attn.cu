@@ -170,26 +170,65 @@ cudaError_t launch_attn_simt(const Geo& g, bool is_bf16, const AttnArgs& a, cuda
 
 // ===========================================================================
 // tcgen05 path (bf16, bs == 128)
+//
+// One CTA owns two query tiles (two consecutive tiles of the tile order).
+// Warps 0-3 run the softmax of tile 0 and warps 4-7 that of tile 1, warp 8
+// issues the TMA loads and warp 9 the MMAs.  While one softmax warpgroup
+// works on its S, the tensor core runs the other tile's O += P V and its next
+// S = Q K^T, so MMAs and exponentials overlap.  TMEM (512 columns): S of tile
+// x at 128x, O of tile x at 256 + 128x; P (bf16 pairs, even key in the low
+// half) overwrites the first 64 columns of S and is the A operand of the PV
+// MMA.  K and V tiles stream through one ring of shared-memory slots in the
+// order the MMA warp consumes them:
+//   S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) | PV0(1) S0(2) PV1(1) S1(2) | ...
+// A commit after S_x(s) covers every MMA issued before it, so when the
+// softmax warps see S_x(s) the previous PV of the tile is complete and O_x
+// may be rescaled in place.  The running max is only moved (and O rescaled)
+// when it grows by more than 8 in log2 units; until then the exponentials
+// are taken against the stale max (values stay below 2^8).
 // ===========================================================================
 template <int HD>
 struct TcLayout {
   static constexpr int kTile = 128 * HD * 2;   // one 128-row bf16 tile
   static constexpr int kPanel = 128 * 128;     // 128 rows x 128 bytes (one TMA box)
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTile;        // 2 stages
-  static constexpr int kV = kK + 2 * kTile;    // 2 stages
-  static constexpr int kP = kV + 2 * kTile;    // 128 x 128 bf16, 2 panels
-  static constexpr int kBars = kP + 2 * kPanel;
-  // 0 q_full, 1-2 k_full, 3-4 v_full, 5-6 kv_empty, 7 s_full, 8 p_full, 9 o_done, 10 final
-  static constexpr int kNumBars = 11;
+  static constexpr int kStages = HD == 128 ? 4 : 8;
+  static constexpr int kQ = 0;                 // two query tiles
+  static constexpr int kRing = kQ + 2 * kTile; // K/V ring
+  static constexpr int kBars = kRing + kStages * kTile;
+  // q_full[2], kv_full[kStages], kv_empty[kStages], s_full[2], p_full[2], o_final[2], final
+  static constexpr int kBarQ = 0, kBarFull = 2, kBarEmpty = 2 + kStages, kBarS = 2 + 2 * kStages,
+                       kBarP = kBarS + 2, kBarO = kBarP + 2, kBarFinal = kBarO + 2;
+  static constexpr int kNumBars = kBarFinal + 1;
   static constexpr int kTmemSlot = kBars + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
 };
 
-constexpr int kTcThreads = 192;
-constexpr uint32_t kTmemCols = 256;
+constexpr int kTcThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;      // log2 units
+
+// Visits the MMA work of the two tiles in issue order: f(kind, tile, step),
+// kind 0 = S = Q K^T (consumes a K slot), kind 1 = O += P V (a V slot).
+// Stops early and returns false if f does.
+template <class F>
+__device__ __forceinline__ bool for_each_event(int n0, int n1, F&& f) {
+  if (n0 > 0 && !f(0, 0, 0)) return false;
+  if (n1 > 0 && !f(0, 1, 0)) return false;
+  const int rounds = n0 > n1 ? n0 : n1;
+  for (int r = 0; r < rounds; ++r) {
+    if (r < n0) {
+      if (!f(1, 0, r)) return false;
+      if (r + 1 < n0 && !f(0, 0, r + 1)) return false;
+    }
+    if (r < n1) {
+      if (!f(1, 1, r)) return false;
+      if (r + 1 < n1 && !f(0, 1, r + 1)) return false;
+    }
+  }
+  return true;
+}
 
 template <int HD>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -199,34 +238,46 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_addr(sm);
-  const uint32_t sQ = sb + L::kQ, sK = sb + L::kK, sV = sb + L::kV, sP = sb + L::kP;
+  const uint32_t sRing = sb + L::kRing;
   const uint32_t bar0 = sb + L::kBars;
-  const uint32_t bar_q = bar0, bar_s = bar0 + 7 * 8, bar_p = bar0 + 8 * 8, bar_o = bar0 + 9 * 8;
-  const uint32_t bar_final = bar0 + 10 * 8;
-  auto bar_k = [&](int st) { return bar0 + (1 + st) * 8; };
-  auto bar_v = [&](int st) { return bar0 + (3 + st) * 8; };
-  auto bar_e = [&](int st) { return bar0 + (5 + st) * 8; };
+  auto bar = [&](int x) { return bar0 + 8u * (uint32_t)x; };
   volatile int* abort = reinterpret_cast<volatile int*>(sm + L::kAbort);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int b, h, i;
-  decode_tile(g, blockIdx.x, b, h, i);
-  const long long bh = (long long)b * g.Hd + h;
   const int nbk = g.nb + g.nb_text;
-  const bool dense_row = i >= g.nb;
-  const int n = list_length(g, a, bh, i);
-  const int32_t* list = a.idx + (bh * g.nb + (dense_row ? 0 : i)) * a.kmax;
-  auto block_at = [&](int s) -> int {
-    const int j = dense_row ? s : __ldg(list + s);
+  const int n_tiles = g.B * g.Hd * nbk;
+
+  // The two query tiles of this CTA (held in scalars: a runtime-indexed array
+  // would live in local memory).
+  int i0 = -1, i1 = -1, n0 = 0, n1 = 0;
+  long long bh0 = 0, bh1 = 0;
+  {
+    int b, h, i;
+    if (2 * (int)blockIdx.x < n_tiles) {
+      decode_tile(g, 2 * blockIdx.x, b, h, i);
+      i0 = i; bh0 = (long long)b * g.Hd + h; n0 = list_length(g, a, bh0, i);
+    }
+    if (2 * (int)blockIdx.x + 1 < n_tiles) {
+      decode_tile(g, 2 * blockIdx.x + 1, b, h, i);
+      i1 = i; bh1 = (long long)b * g.Hd + h; n1 = list_length(g, a, bh1, i);
+    }
+  }
+  const int32_t* list0 = a.idx + (bh0 * g.nb + (i0 >= 0 && i0 < g.nb ? i0 : 0)) * a.kmax;
+  const int32_t* list1 = a.idx + (bh1 * g.nb + (i1 >= 0 && i1 < g.nb ? i1 : 0)) * a.kmax;
+  // Key block of step s of tile x; -1 for an out-of-range list entry.
+  auto block_at = [&](int x, int s) -> int {
+    const int i = x ? i1 : i0;
+    const int j = i >= g.nb ? s : __ldg((x ? list1 : list0) + s);
     return (j >= 0 && j < nbk) ? j : -1;
   };
 
   if (threadIdx.x == 0) {
-    for (int x = 0; x < L::kNumBars; ++x) mbar_init(bar0 + 8 * x, x == 8 ? 128 : 1);
+    for (int x = 0; x < L::kNumBars; ++x)
+      mbar_init(bar(x), (x == L::kBarP || x == L::kBarP + 1) ? 128u : 1u);
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(sb + L::kTmemSlot, kTmemCols);
     tmem_relinquish();
   }
@@ -234,196 +285,201 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + L::kTmemSlot);
-  const uint32_t tS = tmem, tO = tmem + 128;
   constexpr uint32_t kTileBytes = L::kTile;
   constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
   constexpr uint32_t idesc_o = idesc_bf16_f32(128, HD, 0, 1);
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const int qrow = (int)((bh * nbk + i) * 128);
-      mbar_arrive_expect_tx(bar_q, kTileBytes);
-      for (int p = 0; p < HD / 64; ++p) tma_load_2d(sQ + p * L::kPanel, &tq, 64 * p, qrow, bar_q);
-      int it = 0;
-      bool bad = false;
-      for (int s = 0; s < n; ++s) {
-        const int j = block_at(s);
-        if (j < 0) { bad = true; continue; }
-        const int st = it & 1;
-        if (it >= 2 && !mbar_wait(bar_e(st), ((it >> 1) - 1) & 1, abort)) break;
-        const int krow = (int)((bh * nbk + j) * 128);
-        mbar_arrive_expect_tx(bar_k(st), kTileBytes);
+      for (int x = 0; x < 2; ++x) {
+        if ((x ? n1 : n0) == 0) continue;
+        const int qrow = (int)(((x ? bh1 : bh0) * nbk + (x ? i1 : i0)) * 128);
+        mbar_arrive_expect_tx(bar(L::kBarQ + x), kTileBytes);
         for (int p = 0; p < HD / 64; ++p)
-          tma_load_2d(sK + st * kTileBytes + p * L::kPanel, &tk, 64 * p, krow, bar_k(st));
-        mbar_arrive_expect_tx(bar_v(st), kTileBytes);
-        for (int p = 0; p < HD / 64; ++p)
-          tma_load_2d(sV + st * kTileBytes + p * L::kPanel, &tv, 64 * p, krow, bar_v(st));
-        ++it;
+          tma_load_2d(sb + L::kQ + x * kTileBytes + p * L::kPanel, &tq, 64 * p, qrow, bar(L::kBarQ + x));
       }
+      int pos = 0;
+      bool bad = false;
+      for_each_event(n0, n1, [&](int kind, int x, int s) -> bool {
+        int j = block_at(x, s);
+        if (j < 0) { bad = true; j = 0; }   // load some tile; the softmax masks the step
+        const int slot = pos % L::kStages;
+        if (pos >= L::kStages &&
+            !mbar_wait(bar(L::kBarEmpty + slot), ((pos / L::kStages) - 1) & 1, abort))
+          return false;
+        const int row = (int)(((x ? bh1 : bh0) * nbk + j) * 128);
+        const uint32_t dst = sRing + slot * kTileBytes;
+        mbar_arrive_expect_tx(bar(L::kBarFull + slot), kTileBytes);
+        for (int p = 0; p < HD / 64; ++p)
+          tma_load_2d(dst + p * L::kPanel, kind == 0 ? &tk : &tv, 64 * p, row, bar(L::kBarFull + slot));
+        ++pos;
+        return true;
+      });
       if (bad) set_status(a.status, 6);
       // Never leave the CTA with a copy in flight: wait for the last loads.
-      mbar_wait(bar_q, 0, abort);
-      for (int x = (it >= 2 ? it - 2 : 0); x < it; ++x) {
-        mbar_wait(bar_k(x & 1), (x >> 1) & 1, abort);
-        mbar_wait(bar_v(x & 1), (x >> 1) & 1, abort);
-      }
+      for (int x = 0; x < 2; ++x)
+        if ((x ? n1 : n0) > 0) mbar_wait(bar(L::kBarQ + x), 0, abort);
+      for (int p = (pos > L::kStages ? pos - L::kStages : 0); p < pos; ++p)
+        mbar_wait(bar(L::kBarFull + p % L::kStages), (p / L::kStages) & 1, abort);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int it = 0;
-      bool ok = mbar_wait(bar_q, 0, abort);
+      bool ok = true;
+      for (int x = 0; x < 2; ++x)
+        if ((x ? n1 : n0) > 0 && !mbar_wait(bar(L::kBarQ + x), 0, abort)) ok = false;
       tc_fence_after();
-      auto issue_pv = [&](int x) -> bool {
-        const int st = x & 1;
-        if (!mbar_wait(bar_p, x & 1, abort)) return false;
-        if (!mbar_wait(bar_v(st), (x >> 1) & 1, abort)) return false;
-        tc_fence_after();
+      int pos = 0;
+      if (ok) {
+        for_each_event(n0, n1, [&](int kind, int x, int s) -> bool {
+          const int slot = pos % L::kStages;
+          if (!mbar_wait(bar(L::kBarFull + slot), (pos / L::kStages) & 1, abort)) return false;
+          tc_fence_after();
+          const uint32_t src = sRing + slot * kTileBytes;
+          const uint32_t tS = tmem + 128u * x;
+          if (kind == 0) {
+            const uint32_t sQ = sb + L::kQ + x * kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = smem_desc_sw128(sP + (kk >> 2) * L::kPanel + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sV + st * kTileBytes + kk * 2048, L::kPanel, 1024);
-          mma_bf16_ss(tO, ad, bd, idesc_o, (x > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(bar_o);
-        tc_commit(bar_e(st));
-        return true;
-      };
-      for (int s = 0; s < n && ok; ++s) {
-        if (block_at(s) < 0) continue;
-        const int st = it & 1;
-        if (!mbar_wait(bar_k(st), (it >> 1) & 1, abort)) { ok = false; break; }
-        tc_fence_after();
-        if (it > 0 && !issue_pv(it - 1)) { ok = false; break; }
+            for (int kk = 0; kk < HD / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * L::kPanel + (kk & 3) * 32;
+              mma_bf16_ss(tS, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(src + off, 16, 1024),
+                          idesc_s, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(bar(L::kBarS + x));
+          } else {
+            if (!mbar_wait(bar(L::kBarP + x), s & 1, abort)) return false;
+            tc_fence_after();
+            const uint32_t tO = tmem + 256u + 128u * x;
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kPanel + (kk & 3) * 32;
-          const uint64_t ad = smem_desc_sw128(sQ + off, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sK + st * kTileBytes + off, 16, 1024);
-          mma_bf16_ss(tS, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(bar_s);
-        ++it;
+            for (int kk = 0; kk < 8; ++kk)
+              mma_bf16_ts(tO, tS + 8u * kk, smem_desc_sw128(src + kk * 2048, L::kPanel, 1024), idesc_o,
+                          (s > 0 || kk > 0) ? 1u : 0u);
+            if (s == (x ? n1 : n0) - 1) tc_commit(bar(L::kBarO + x));
+          }
+          tc_commit(bar(L::kBarEmpty + slot));
+          ++pos;
+          return true;
+        });
       }
-      if (ok && it > 0) issue_pv(it - 1);
       // Every MMA issued must be complete before TMEM is released.
-      tc_commit(bar_final);
-      mbar_wait(bar_final, 0, abort);
+      tc_commit(bar(L::kBarFinal));
+      mbar_wait(bar(L::kBarFinal), 0, abort);
     }
   } else {
-    // ------------------------------------------------------------ softmax warps 0-3
-    const int r = warp * 32 + lane;                      // query row = TMEM lane
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    float m = -INFINITY, l = 0.f;
-    int it = 0;
-    bool ok = true;
-    for (int s = 0; s < n; ++s) {
-      const int j = block_at(s);
-      if (j < 0) continue;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_s, it & 1, abort))) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[128];
-      TMEM_LD32(tS + lane_off + 0, (sr + 0));
-      TMEM_LD32(tS + lane_off + 32, (sr + 32));
-      TMEM_LD32(tS + lane_off + 64, (sr + 64));
-      TMEM_LD32(tS + lane_off + 96, (sr + 96));
-      TMEM_LD_WAIT((sr + 0));
-      TMEM_LD_WAIT((sr + 32));
-      TMEM_LD_WAIT((sr + 64));
-      TMEM_LD_WAIT((sr + 96));
-      const uint4 mw = __ldg(reinterpret_cast<const uint4*>(a.masks) + j);
-      if ((mw.x & mw.y & mw.z & mw.w) != 0xffffffffu) {
-        const uint32_t w4[4] = {mw.x, mw.y, mw.z, mw.w};
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (!((w4[c >> 5] >> (c & 31)) & 1u)) sr[c] = __float_as_uint(-INFINITY);
-      }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
-      const float m_new = fmaxf(m, mx * a.scale_log2);
-      const float corr = fast_ex2(m - m_new);
-      float rowsum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const float p = fast_ex2(fmaf(__uint_as_float(sr[c]), a.scale_log2, -m_new));
-        rowsum += p;
-        sr[c] = __float_as_uint(p);
-      }
-      l = l * corr + rowsum;
-      m = m_new;
-      if (it > 0) {
-        // PV of the previous step must be done: P buffer free, O stable.
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_o, (it - 1) & 1, abort))) { ok = false; break; }
+    // ------------------------------------------------------------ softmax warpgroups
+    const int x = warp >> 2, wq = warp & 3;
+    const int r = wq * 32 + lane;                        // query row = TMEM lane
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + 128u * x + lane_off;
+    const uint32_t tO = tmem + 256u + 128u * x + lane_off;
+    const int n = x ? n1 : n0;
+    const int qi = x ? i1 : i0;
+    const long long qbh = x ? bh1 : bh0;
+    if (qi >= 0) {
+      float m_run = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int s = 0; s < n; ++s) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + x), s & 1, abort))) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, corr != 1.f)) {
+        uint32_t sr[128];
+        TMEM_LD32(tS + 0, (sr + 0));
+        TMEM_LD32(tS + 32, (sr + 32));
+        TMEM_LD32(tS + 64, (sr + 64));
+        TMEM_LD32(tS + 96, (sr + 96));
+        TMEM_LD_WAIT((sr + 0));
+        TMEM_LD_WAIT((sr + 32));
+        TMEM_LD_WAIT((sr + 64));
+        TMEM_LD_WAIT((sr + 96));
+        const int j = block_at(x, s);
+        uint4 mw = make_uint4(0u, 0u, 0u, 0u);
+        if (j >= 0) mw = __ldg(reinterpret_cast<const uint4*>(a.masks) + j);
+        if ((mw.x & mw.y & mw.z & mw.w) != 0xffffffffu) {
+          const uint32_t w4[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (!((w4[c >> 5] >> (c & 31)) & 1u)) sr[c] = __float_as_uint(-INFINITY);
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+        const float m_cand = mx * a.scale_log2;
+        const bool need = m_cand > m_run + kRescaleThreshold;
+        const bool any_need = __any_sync(0xffffffffu, need);
+        float scale = 1.f;
+        if (any_need) {
+          const float m_new = need ? m_cand : m_run;
+          scale = need ? fast_ex2(m_run - m_new) : 1.f;
+          l *= scale;
+          m_run = m_new;
+        }
+        const float m_use = m_run == -INFINITY ? 0.f : m_run;
+        float rowsum = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float p0 = fast_ex2(fmaf(__uint_as_float(sr[2 * c]), a.scale_log2, -m_use));
+          const float p1 = fast_ex2(fmaf(__uint_as_float(sr[2 * c + 1]), a.scale_log2, -m_use));
+          rowsum += p0 + p1;
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        l += rowsum;
+        TMEM_ST32(tS + 0, (pk + 0));
+        TMEM_ST32(tS + 32, (pk + 32));
+        // O of the previous steps is complete (this S was committed after the
+        // previous PV), so it can be rescaled before this step's PV is issued.
+        if (any_need && s > 0) {
 #pragma unroll
           for (int c0 = 0; c0 < HD; c0 += 32) {
             uint32_t orr[32];
-            TMEM_LD32(tO + lane_off + c0, orr);
+            TMEM_LD32(tO + c0, orr);
             TMEM_LD_WAIT(orr);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * corr);
-            TMEM_ST32(tO + lane_off + c0, orr);
+            for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * scale);
+            TMEM_ST32(tO + c0, orr);
           }
-          tmem_st_wait();
         }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(L::kBarP + x));
       }
-      // P row -> shared memory, K-major with the 128-byte swizzle.
-#pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8) {
-        uint4 v;
-        v.x = pack_bf16x2(__uint_as_float(sr[8 * c8 + 0]), __uint_as_float(sr[8 * c8 + 1]));
-        v.y = pack_bf16x2(__uint_as_float(sr[8 * c8 + 2]), __uint_as_float(sr[8 * c8 + 3]));
-        v.z = pack_bf16x2(__uint_as_float(sr[8 * c8 + 4]), __uint_as_float(sr[8 * c8 + 5]));
-        v.w = pack_bf16x2(__uint_as_float(sr[8 * c8 + 6]), __uint_as_float(sr[8 * c8 + 7]));
-        const uint32_t addr = sP + (c8 >> 3) * L::kPanel + r * 128 + ((((c8 & 7) ^ (r & 7))) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
-                     "r"(v.z), "r"(v.w)
-                     : "memory");
+      // ---- epilogue: O / l -> blocked output row
+      if (ok && n > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarO + x), 0, abort));
+        tc_fence_after();
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar_p);
-      ++it;
-    }
-    // ---- epilogue: O / l -> blocked output row
-    if (ok && it > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (it - 1) & 1, abort));
-      tc_fence_after();
-    }
-    const uint4 qm = __ldg(reinterpret_cast<const uint4*>(a.masks) + i);
-    const uint32_t qw4[4] = {qm.x, qm.y, qm.z, qm.w};
-    const bool row_valid = ((qw4[r >> 5] >> (r & 31)) & 1u) && ok && it > 0;
-    const float inv = (row_valid && l > 0.f) ? 1.f / l : 0.f;
-    uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) +
-                                           ((bh * nbk + i) * 128 + r) * HD);
+      const uint4 qm = __ldg(reinterpret_cast<const uint4*>(a.masks) + qi);
+      const uint32_t qw4[4] = {qm.x, qm.y, qm.z, qm.w};
+      const bool row_valid = ((qw4[r >> 5] >> (r & 31)) & 1u) && ok && n > 0;
+      const float inv = (row_valid && l > 0.f) ? 1.f / l : 0.f;
+      uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) +
+                                             ((qbh * nbk + qi) * 128 + r) * HD);
 #pragma unroll
-    for (int c0 = 0; c0 < HD; c0 += 32) {
-      uint32_t orr[32];
-      if (ok && it > 0) {
-        TMEM_LD32(tO + lane_off + c0, orr);
-        TMEM_LD_WAIT(orr);
-      } else {
+      for (int c0 = 0; c0 < HD; c0 += 32) {
+        uint32_t orr[32];
+        if (ok && n > 0) {
+          TMEM_LD32(tO + c0, orr);
+          TMEM_LD_WAIT(orr);
+        } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) orr[c] = 0u;
-      }
+          for (int c = 0; c < 32; ++c) orr[c] = 0u;
+        }
 #pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8) {
-        uint4 v;
-        v.x = pack_bf16x2(__uint_as_float(orr[8 * c8 + 0]) * inv, __uint_as_float(orr[8 * c8 + 1]) * inv);
-        v.y = pack_bf16x2(__uint_as_float(orr[8 * c8 + 2]) * inv, __uint_as_float(orr[8 * c8 + 3]) * inv);
-        v.z = pack_bf16x2(__uint_as_float(orr[8 * c8 + 4]) * inv, __uint_as_float(orr[8 * c8 + 5]) * inv);
-        v.w = pack_bf16x2(__uint_as_float(orr[8 * c8 + 6]) * inv, __uint_as_float(orr[8 * c8 + 7]) * inv);
-        orow[c0 / 8 + c8] = v;
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(orr[8 * c8 + 0]) * inv, __uint_as_float(orr[8 * c8 + 1]) * inv);
+          v.y = pack_bf16x2(__uint_as_float(orr[8 * c8 + 2]) * inv, __uint_as_float(orr[8 * c8 + 3]) * inv);
+          v.z = pack_bf16x2(__uint_as_float(orr[8 * c8 + 4]) * inv, __uint_as_float(orr[8 * c8 + 5]) * inv);
+          v.w = pack_bf16x2(__uint_as_float(orr[8 * c8 + 6]) * inv, __uint_as_float(orr[8 * c8 + 7]) * inv);
+          orow[c0 / 8 + c8] = v;
+        }
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -438,17 +494,18 @@ cudaError_t launch_attn_tc(const Geo& g, const AttnArgs& a, const CUtensorMap& t
                            const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
   const int tiles = g.B * g.Hd * (g.nb + g.nb_text);
   if (tiles == 0) return cudaSuccess;
+  const int ctas = (tiles + 1) / 2;
   cudaError_t e;
   if (g.D == 128) {
     const int smem = TcLayout<128>::kAlloc;
     e = cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_tc_kernel<128><<<tiles, kTcThreads, smem, st>>>(g, a, tq, tk, tv);
+    attn_tc_kernel<128><<<ctas, kTcThreads, smem, st>>>(g, a, tq, tk, tv);
   } else {
     const int smem = TcLayout<64>::kAlloc;
     e = cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_tc_kernel<64><<<tiles, kTcThreads, smem, st>>>(g, a, tq, tk, tv);
+    attn_tc_kernel<64><<<ctas, kTcThreads, smem, st>>>(g, a, tq, tk, tv);
   }
   return cudaGetLastError();
 }
