@@ -184,6 +184,10 @@ def run_ours(args, rank, world, local):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300),
                                 device_id=dev)
     w = synthetic.workload(args.workload)
+    if args.heads:
+        reps = args.heads // len(w.params) + 1
+        w.Hd, w.params = args.heads, (w.params * reps)[:args.heads]
+        w.name = f"{w.name}_{args.heads}heads"
     q, k, v = synthetic.make_qkv(w)
     plan = bsa.plan_for(w, dev)
     kmax = plan.kmax_for(w.mode, w.params)
@@ -421,6 +425,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the workload's head count (smaller profiling cases)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
     rank, world, local = dist_env()

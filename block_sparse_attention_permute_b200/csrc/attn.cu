@@ -205,7 +205,18 @@ struct TcLayout {
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
 };
 
-constexpr int kTcThreads = 320;
+// Warps 0-3 and 4-7: softmax of tile 0 and tile 1; warp 8: TMA producer;
+// warp 9: MMA issuer; warps 10-11 only complete the third warpgroup so that
+// registers can be moved between warpgroups with setmaxnreg.
+constexpr int kTcThreads = 384;
+// Registers per thread: the launch gives every thread kRegsLaunch; then the
+// producer/MMA warpgroup drops to kRegsSmall and the two softmax warpgroups
+// rise to kRegsSoftmax.  2 * 128 * kRegsSoftmax + 128 * kRegsSmall must not
+// exceed 384 * kRegsLaunch (checked below).
+constexpr int kRegsLaunch = 168, kRegsSoftmax = 216, kRegsSmall = 72;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsSmall <= kTcThreads * kRegsLaunch,
+              "register split exceeds the launch allocation");
+constexpr int kExpFmaPairsPer8 = 0;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;      // log2 units
 
@@ -288,8 +299,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr uint32_t kTileBytes = L::kTile;
   constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
   constexpr uint32_t idesc_o = idesc_bf16_f32(128, HD, 0, 1);
-
-  if (warp == 8) {
+  if (warp >= 8) {
+   // ============================================================ warpgroup 2
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSmall));
+   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       for (int x = 0; x < 2; ++x) {
@@ -366,7 +379,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_commit(bar(L::kBarFinal));
       mbar_wait(bar(L::kBarFinal), 0, abort);
     }
+   }
   } else {
+    // ============================================================ warpgroups 0-1
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ------------------------------------------------------------ softmax warpgroups
     const int x = warp >> 2, wq = warp & 3;
     const int r = wq * 32 + lane;                        // query row = TMEM lane
@@ -379,7 +395,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (qi >= 0) {
       float m_run = -INFINITY, l = 0.f;
       bool ok = true;
+      // Block id and slot-validity mask of the next step, loaded one step
+      // ahead so that their latency hides behind the wait for S.
+      int j_next = n > 0 ? block_at(x, 0) : -1;
+      uint4 mw_next = j_next >= 0 ? __ldg(reinterpret_cast<const uint4*>(a.masks) + j_next)
+                                  : make_uint4(0u, 0u, 0u, 0u);
       for (int s = 0; s < n; ++s) {
+        const uint4 mw = mw_next;
+        if (s + 1 < n) {
+          j_next = block_at(x, s + 1);
+          mw_next = j_next >= 0 ? __ldg(reinterpret_cast<const uint4*>(a.masks) + j_next)
+                                : make_uint4(0u, 0u, 0u, 0u);
+        }
         if (!__all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + x), s & 1, abort))) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[128];
@@ -391,18 +418,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         TMEM_LD_WAIT((sr + 32));
         TMEM_LD_WAIT((sr + 64));
         TMEM_LD_WAIT((sr + 96));
-        const int j = block_at(x, s);
-        uint4 mw = make_uint4(0u, 0u, 0u, 0u);
-        if (j >= 0) mw = __ldg(reinterpret_cast<const uint4*>(a.masks) + j);
         if ((mw.x & mw.y & mw.z & mw.w) != 0xffffffffu) {
           const uint32_t w4[4] = {mw.x, mw.y, mw.z, mw.w};
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (!((w4[c >> 5] >> (c & 31)) & 1u)) sr[c] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
+        // Row max over 8 independent partial maxima (short dependency chains).
+        float mp[8];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+        for (int k = 0; k < 8; ++k) mp[k] = __uint_as_float(sr[k]);
+#pragma unroll
+        for (int c = 8; c < 128; ++c) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(sr[c]));
+        const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                               fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
         const float m_cand = mx * a.scale_log2;
         const bool need = m_cand > m_run + kRescaleThreshold;
         const bool any_need = __any_sync(0xffffffffu, need);
@@ -414,16 +443,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           m_run = m_new;
         }
         const float m_use = m_run == -INFINITY ? 0.f : m_run;
-        float rowsum = 0.f;
+        const float2 sl2 = make_float2(a.scale_log2, a.scale_log2);
+        const float2 neg_m = make_float2(-m_use, -m_use);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
         uint32_t pk[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float p0 = fast_ex2(fmaf(__uint_as_float(sr[2 * c]), a.scale_log2, -m_use));
-          const float p1 = fast_ex2(fmaf(__uint_as_float(sr[2 * c + 1]), a.scale_log2, -m_use));
-          rowsum += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
+          const float2 t = fma2(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])),
+                                sl2, neg_m);
+          // kExpFmaPairsPer8 of every 8 pairs take the FMA-pipe exponential.
+          const float2 p = ((c & 7) < kExpFmaPairsPer8) ? exp2_fma2(t)
+                                                        : make_float2(fast_ex2(t.x), fast_ex2(t.y));
+          acc[c & 3] = add2(acc[c & 3], p);
+          pk[c] = pack_bf16x2(p.x, p.y);
         }
-        l += rowsum;
+        const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
+        const float2 a03 = add2(a01, a23);
+        l += a03.x + a03.y;
         TMEM_ST32(tS + 0, (pk + 0));
         TMEM_ST32(tS + 32, (pk + 32));
         // O of the previous steps is complete (this S was committed after the
@@ -495,7 +532,13 @@ cudaError_t launch_attn_tc(const Geo& g, const AttnArgs& a, const CUtensorMap& t
   const int tiles = g.B * g.Hd * (g.nb + g.nb_text);
   if (tiles == 0) return cudaSuccess;
   const int ctas = (tiles + 1) / 2;
-  cudaError_t e;
+  // The setmaxnreg split assumes the launch gives every thread exactly
+  // kRegsLaunch registers; refuse to launch a build where that is not so.
+  cudaFuncAttributes attr;
+  cudaError_t e = g.D == 128 ? cudaFuncGetAttributes(&attr, attn_tc_kernel<128>)
+                             : cudaFuncGetAttributes(&attr, attn_tc_kernel<64>);
+  if (e != cudaSuccess) return e;
+  if (attr.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
   if (g.D == 128) {
     const int smem = TcLayout<128>::kAlloc;
     e = cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
