@@ -2,16 +2,19 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-A step is one bsa_forward (permute -> select -> attention -> unpermute) over
-one batch of synthetic input already resident in HBM.  Default workload: the
+A step is one bsa_forward over one batch of synthetic input already resident
+in HBM: on the tensor-core plans that is centroids -> selection -> attention
+with the layout transform (permute) and its inverse fused into the
+attention's TMA loads and stores.  Default workload: the
 HunyuanVideo 720p 61-frame shape (16x45x80 latent grid + 256 text tokens,
 24 heads, head_dim 128, bf16, 1x8x16 blocks, density 0.15).
 
 Printed: one JSON line on rank 0.  value = effective TFLOP/s of the whole job
 = 4 x selected valid (query, key) pairs x head_dim (summed over heads and
 ranks) / max-over-ranks device time.  Per-phase times come from a second loop
-that issues the same four calls separately, with CUDA events on the
-launching stream.  Under torchrun every rank runs its own replica of the
+that issues bsa_forward's calls separately, with CUDA events on the launching
+stream; a third loop times the unfused pipeline (bsa_permute_qkv,
+selection, bsa_attention on the blocked layout, bsa_unpermute) for reference.  Under torchrun every rank runs its own replica of the
 workload (weak scaling, no collective on the data path).
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
@@ -232,33 +235,47 @@ def run_ours(args, rank, world, local):
     step_ms = ev0.elapsed_time(ev1) / args.steps
     clocks = clk.summary()
 
-    # ---- phase loop: the same four calls, separately timed
-    qb, kb, vb, ob = (torch.empty(plan.blk_shape, dtype=plan.dtype, device=dev) for _ in range(4))
-    qc, kc = (torch.empty(plan.cent_shape, dtype=torch.float32, device=dev) for _ in range(2))
-    names = ["permute", "select", "attention", "unpermute"]
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    calls = [
-        lambda: L.bsa_permute_qkv(plan._h, P(qd), P(kd), P(vd), P(qb), P(kb), P(vb), P(qc), P(kc),
-                                  bsa._stream(dev)),
-        lambda: L.bsa_select_centroids(plan._h, P(qc), P(kc), w.mode, params, kmax, P(idx), P(cnt),
-                                       None, bsa._stream(dev)),
-        lambda: L.bsa_attention(plan._h, P(qb), P(kb), P(vb), P(idx), P(cnt), kmax, P(ob), None,
-                                bsa._stream(dev)),
-        lambda: L.bsa_unpermute(plan._h, P(ob), P(out), bsa._stream(dev)),
-    ]
-    for _ in range(args.warmup):
-        for c in calls:
-            bsa._check(c())
-    barrier()
-    for s in range(args.steps):
-        evs[s][0].record(stream)
-        for ci, c in enumerate(calls):
-            bsa._check(c())
-            evs[s][ci + 1].record(stream)
-    barrier()
-    plan.check_status()
-    phase_ms = {n: sum(evs[s][ci].elapsed_time(evs[s][ci + 1]) for s in range(args.steps)) / args.steps
+    # ---- phase loops (CUDA events on the launching stream)
+    def time_phases(names, calls):
+        for _ in range(args.warmup):
+            for c in calls:
+                bsa._check(c())
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+               for _ in range(args.steps)]
+        barrier()
+        for st_i in range(args.steps):
+            evs[st_i][0].record(stream)
+            for ci, c in enumerate(calls):
+                bsa._check(c())
+                evs[st_i][ci + 1].record(stream)
+        barrier()
+        plan.check_status()
+        return {n: sum(evs[si][ci].elapsed_time(evs[si][ci + 1]) for si in range(args.steps)) / args.steps
                 for ci, n in enumerate(names)}
+
+    qc, kc = (torch.empty(plan.cent_shape, dtype=torch.float32, device=dev) for _ in range(2))
+    S = lambda: bsa._stream(dev)
+    if plan.info.attn_path == 1:
+        # what bsa_forward runs on this plan: the layout transform is fused into the attention
+        fused = time_phases(
+            ["centroids", "select", "attention"],
+            [lambda: L.bsa_centroids(plan._h, P(qd), P(kd), P(qc), P(kc), S()),
+             lambda: L.bsa_select_centroids(plan._h, P(qc), P(kc), w.mode, params, kmax, P(idx),
+                                            P(cnt), None, S()),
+             lambda: L.bsa_attention_orig(plan._h, P(qd), P(kd), P(vd), P(idx), P(cnt), kmax, P(out),
+                                          None, S())])
+    else:
+        fused = None
+    qb, kb, vb, ob = (torch.empty(plan.blk_shape, dtype=plan.dtype, device=dev) for _ in range(4))
+    unfused = time_phases(
+        ["permute", "select", "attention", "unpermute"],
+        [lambda: L.bsa_permute_qkv(plan._h, P(qd), P(kd), P(vd), P(qb), P(kb), P(vb), P(qc), P(kc), S()),
+         lambda: L.bsa_select_centroids(plan._h, P(qc), P(kc), w.mode, params, kmax, P(idx), P(cnt),
+                                        None, S()),
+         lambda: L.bsa_attention(plan._h, P(qb), P(kb), P(vb), P(idx), P(cnt), kmax, P(ob), None, S()),
+         lambda: L.bsa_unpermute(plan._h, P(ob), P(out), S())])
+    del qb, kb, vb, ob
+    phase_ms = fused if fused is not None else unfused
 
     # ---- end to end: pinned host buffers, copies inside the timed region
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
@@ -316,13 +333,17 @@ def run_ours(args, rank, world, local):
             "selected_pairs": pairs,
         },
         "phases_ms": {n: round(t, 4) for n, t in phase_ms.items()},
+        "phases_ms_unfused": {n: round(t, 4) for n, t in unfused.items()},
         "attn_tflops": round(attn_tf, 2),
         "attn_frac_of_peak": round(attn_tf / peak_tf, 4),
         "permute_select_share_of_attn": round(
-            (phase_ms["permute"] + phase_ms["select"]) / phase_ms["attention"], 4),
+            (phase_ms.get("centroids", phase_ms.get("permute", 0.0)) + phase_ms["select"])
+            / phase_ms["attention"], 4),
+        "permute_select_share_of_attn_unfused": round(
+            (unfused["permute"] + unfused["select"]) / unfused["attention"], 4),
         "roofline": {
             "bound": "tensor",
-            "kernel": "attn_tc_kernel",
+            "kernel": "attn_tc_kernel<128, original layout>" if plan.info.attn_path == 1 else "attn_simt_kernel",
             "achieved": round(attn_tf, 2),
             "peak": peak_tf,
             "peak_source": f"{peak_src} bf16_tflops_sustained (MEASURED_PEAKS.json)",
@@ -333,7 +354,7 @@ def run_ours(args, rank, world, local):
         "e2e": {"value": round(job_tflops(world, flops, e2e_ms), 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": (3 if plan.info.attn_path == 1 else 4) * args.steps,
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -69,6 +69,8 @@ def load():
         "bsa_permute": [P, P, P, P, P],
         "bsa_permute_qkv": [P] * 10,
         "bsa_unpermute": [P, P, P, P],
+        "bsa_centroids": [P, P, P, P, P, P],
+        "bsa_attention_orig": [P, P, P, P, P, P, I, P, P, P],
         "bsa_select": [P, P, P, I, P, I, P, P, P, P, Z, P],
         "bsa_select_centroids": [P, P, P, I, P, I, P, P, P, P],
         "bsa_attention": [P, P, P, P, P, P, I, P, P, P],
@@ -189,6 +191,28 @@ class Plan:
         _check(load().bsa_permute_qkv(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(qb), _ptr(kb),
                                       _ptr(vb), _ptr(qc), _ptr(kc), _stream(self.device)))
         return qb, kb, vb, qc, kc
+
+    def centroids(self, q, k):
+        """Q and K block centroids straight from the original layout (bsa_centroids)."""
+        self._check_tensor(q, self.orig_shape, name="q")
+        self._check_tensor(k, self.orig_shape, name="k")
+        qc, kc = (self._new(self.cent_shape, torch.float32) for _ in range(2))
+        _check(load().bsa_centroids(self._h, _ptr(q), _ptr(k), _ptr(qc), _ptr(kc),
+                                    _stream(self.device)))
+        return qc, kc
+
+    def attention_orig(self, q, k, v, idx, cnt, out=None, dev_status=None):
+        """Attention on the original layout; the layout transform is fused (bsa_attention_orig)."""
+        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+            self._check_tensor(t, self.orig_shape, name=n)
+        i = self.info
+        kmax = idx.shape[-1]
+        self._check_tensor(idx, (i.batch, i.heads, i.nb, kmax), torch.int32, "idx")
+        self._check_tensor(cnt, (i.batch, i.heads, i.nb), torch.int32, "cnt")
+        out = self._new(self.orig_shape) if out is None else out
+        _check(load().bsa_attention_orig(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt),
+                                         kmax, _ptr(out), _ptr(dev_status), _stream(self.device)))
+        return out
 
     def unpermute(self, o_blk, out=None):
         self._check_tensor(o_blk, self.blk_shape, name="o_blk")

@@ -118,6 +118,40 @@ bsa_status make_tile_map(CUtensorMap* m, const void* base, long long rows, int D
   return BSA_OK;
 }
 
+CUresult encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                const cuuint64_t* strides, const cuuint32_t* box) {
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+                     dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+// Maps over ONE batch element of an original-layout tensor [Ntot, Hd, D]:
+// video tokens as a 5D tensor (d, head, x, y, t) with box (64, 1, bc, br, bf)
+// (rows land in slot order, the padded part of the box reads zeros); text
+// tokens as a 3D tensor (d, head, token) with box (64, 1, 128).
+bsa_status make_orig_maps(CUtensorMap* video, CUtensorMap* text, const void* x, const Geo& g) {
+  if (encode_fn() == nullptr) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t row = (cuuint64_t)g.D * 2;                    // bytes per (token, head) row
+  const cuuint64_t tok = row * g.Hd;                             // bytes per token
+  cuuint64_t vd[5] = {(cuuint64_t)g.D, (cuuint64_t)g.Hd, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.T};
+  cuuint64_t vs[4] = {row, tok, tok * g.W, tok * g.W * g.H};
+  cuuint32_t vb[5] = {64, 1, (cuuint32_t)g.bc, (cuuint32_t)g.br, (cuuint32_t)g.bf};
+  CUresult r = encode(video, x, 5, vd, vs, vb);
+  if (r != CUDA_SUCCESS) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (video) failed (%d)", (int)r);
+  std::memset(text, 0, sizeof(*text));
+  if (g.n_text > 0) {
+    const char* tbase = reinterpret_cast<const char*>(x) + tok * g.n_video;
+    cuuint64_t td[3] = {(cuuint64_t)g.D, (cuuint64_t)g.Hd, (cuuint64_t)g.n_text};
+    cuuint64_t ts[2] = {row, tok};
+    cuuint32_t tb[3] = {64, 1, 128};
+    r = encode(text, tbase, 3, td, ts, tb);
+    if (r != CUDA_SUCCESS) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (text) failed (%d)", (int)r);
+  }
+  return BSA_OK;
+}
+
 bsa_status run_select(const bsa_plan_s* p, const float* qc, const float* kc, bsa_select_mode mode,
                       const double* param, int kmax, int32_t* idx, int32_t* cnt, float* scores,
                       cudaStream_t st) {
@@ -155,17 +189,83 @@ bsa_status run_attention(const bsa_plan_s* p, const void* q, const void* k, cons
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->g.D));
   cudaError_t e;
   if (p->attn_path == 1) {
-    CUtensorMap tq, tk, tv;
+    bsa::TileMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
     const long long rows = (long long)p->g.B * p->g.Hd * p->g.npad_tot;
     bsa_status s;
-    if ((s = make_tile_map(&tq, q, rows, p->g.D)) != BSA_OK) return s;
-    if ((s = make_tile_map(&tk, k, rows, p->g.D)) != BSA_OK) return s;
-    if ((s = make_tile_map(&tv, v, rows, p->g.D)) != BSA_OK) return s;
-    e = bsa::launch_attn_tc(p->g, a, tq, tk, tv, st);
+    if ((s = make_tile_map(&maps.q, q, rows, p->g.D)) != BSA_OK) return s;
+    if ((s = make_tile_map(&maps.k, k, rows, p->g.D)) != BSA_OK) return s;
+    if ((s = make_tile_map(&maps.v, v, rows, p->g.D)) != BSA_OK) return s;
+    e = bsa::launch_attn_tc(p->g, a, maps, st);
   } else {
     e = bsa::launch_attn_simt(p->g, p->dtype == BSA_BF16, a, st);
   }
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "attention kernel");
+}
+
+bsa_status run_centroids(const bsa_plan_s* p, const void* q, const void* k, float* qc, float* kc,
+                         cudaStream_t st) {
+  // Only the requested tensors are read.
+  bsa::GatherArgs ga;
+  std::memset(&ga, 0, sizeof(ga));
+  if (qc) { ga.src[ga.ntensors] = q; ga.cent[ga.ntensors] = qc; ++ga.ntensors; }
+  if (kc) { ga.src[ga.ntensors] = k; ga.cent[ga.ntensors] = kc; ++ga.ntensors; }
+  if (ga.ntensors == 0 || p->g.nb == 0) return BSA_OK;
+  cudaError_t e = bsa::launch_pool_orig(p->g, p->dtype == BSA_BF16, ga, st);
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "centroid kernel");
+}
+
+// Attention on the original layout, one launch per batch element.
+bsa_status run_attention_orig(const bsa_plan_s* p, const void* q, const void* k, const void* v,
+                              const int32_t* idx, const int32_t* cnt, int kmax, void* o,
+                              int32_t* dev_status, cudaStream_t st) {
+  if (p->attn_path != 1)
+    return fail(BSA_ERR_UNSUPPORTED, "attention on the original layout needs a bf16 plan with 128-token blocks");
+  if (!q || !k || !v || !o) return fail(BSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if (p->g.nb > 0 && (!idx || !cnt)) return fail(BSA_ERR_INVALID_ARG, "NULL index list");
+  if (kmax < 1) return fail(BSA_ERR_INVALID_ARG, "kmax must be >= 1");
+  const size_t per_batch = (size_t)p->g.n_tot * p->g.Hd * p->g.D * 2;
+  Geo g1 = p->g;
+  g1.B = 1;
+  bsa_status s;
+  for (int b = 0; b < p->g.B; ++b) {
+    bsa::TileMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    const char* qb = reinterpret_cast<const char*>(q) + b * per_batch;
+    const char* kb = reinterpret_cast<const char*>(k) + b * per_batch;
+    const char* vb = reinterpret_cast<const char*>(v) + b * per_batch;
+    if ((s = make_orig_maps(&maps.q, &maps.qt, qb, p->g)) != BSA_OK) return s;
+    if ((s = make_orig_maps(&maps.k, &maps.kt, kb, p->g)) != BSA_OK) return s;
+    if ((s = make_orig_maps(&maps.v, &maps.vt, vb, p->g)) != BSA_OK) return s;
+    bsa::AttnArgs a;
+    a.q = qb; a.k = kb; a.v = vb;
+    a.o = reinterpret_cast<char*>(o) + b * per_batch;
+    a.idx = idx + (size_t)b * p->g.Hd * p->g.nb * kmax;
+    a.cnt = cnt + (size_t)b * p->g.Hd * p->g.nb;
+    a.masks = p->d_masks;
+    a.status = dev_status ? dev_status : p->d_status;
+    a.kmax = kmax;
+    a.scale = (float)(1.0 / std::sqrt((double)p->g.D));
+    a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->g.D));
+    cudaError_t e = bsa::launch_attn_tc_orig(g1, a, maps, st);
+    if (e != cudaSuccess) return cuda_fail(e, "attention kernel");
+  }
+  return BSA_OK;
+}
+
+// The fused forward of the tensor-core path: centroids from the original
+// layout, selection, then attention that gathers its tiles from the original
+// layout and scatters the output back.
+bsa_status run_forward_fused(const bsa_plan_s* p, const void* q, const void* k, const void* v,
+                             bsa_select_mode mode, const double* param, int kmax, void* o,
+                             int32_t* idx, int32_t* cnt, float* qc, float* kc,
+                             int32_t* dev_status, cudaStream_t st) {
+  bsa_status s = run_centroids(p, q, k, qc, kc, st);
+  if (s != BSA_OK) return s;
+  if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st)) != BSA_OK) return s;
+  return run_attention_orig(p, q, k, v, idx, cnt, kmax, o, dev_status, st);
 }
 
 }  // namespace
@@ -271,7 +371,9 @@ bsa_status bsa_workspace_size(bsa_plan_t p, int kmax, size_t* select_ws, size_t*
   const size_t lists = round256((size_t)p->g.B * p->g.Hd * p->g.nb * kmax * sizeof(int32_t)) +
                        round256((size_t)p->g.B * p->g.Hd * p->g.nb * sizeof(int32_t));
   if (select_ws) *select_ws = 2 * cent;
-  if (forward_ws) *forward_ws = 4 * round256(blk_bytes(p)) + 2 * cent + lists;
+  // The tensor-core path fuses the layout transform into the attention loads;
+  // the SIMT path stages blocked Q, K, V and O.
+  if (forward_ws) *forward_ws = (p->attn_path == 1 ? 0 : 4 * round256(blk_bytes(p))) + 2 * cent + lists;
   return BSA_OK;
 }
 
@@ -304,6 +406,25 @@ bsa_status bsa_permute_qkv(bsa_plan_t p, const void* q, const void* k, const voi
   a.ntensors = 3;
   cudaError_t e = bsa::launch_permute(p->g, p->dtype == BSA_BF16, a, (cudaStream_t)stream);
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "permute kernel");
+}
+
+bsa_status bsa_centroids(bsa_plan_t p, const void* q, const void* k, float* q_cent, float* k_cent,
+                         void* stream) {
+  bsa_status s = check_plan(p);
+  if (s != BSA_OK) return s;
+  if ((q_cent && !q) || (k_cent && !k)) return fail(BSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  const void* ptrs[4] = {q, k, q_cent, k_cent};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  return run_centroids(p, q, k, q_cent, k_cent, (cudaStream_t)stream);
+}
+
+bsa_status bsa_attention_orig(bsa_plan_t p, const void* q, const void* k, const void* v,
+                              const int32_t* idx, const int32_t* cnt, int kmax, void* o,
+                              int32_t* dev_status, void* stream) {
+  bsa_status s = check_plan(p);
+  if (s != BSA_OK) return s;
+  return run_attention_orig(p, q, k, v, idx, cnt, kmax, o, dev_status, (cudaStream_t)stream);
 }
 
 bsa_status bsa_unpermute(bsa_plan_t p, const void* o_blk, void* o, void* stream) {
@@ -377,7 +498,7 @@ bsa_status bsa_forward(bsa_plan_t p, const void* q, const void* k, const void* v
     return fail(BSA_ERR_WORKSPACE, "forward needs %zu bytes of workspace, got %zu", need_ws, ws_bytes);
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(BSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   char* w = reinterpret_cast<char*>(ws);
-  const size_t tb = round256(blk_bytes(p)), cb = round256(cent_bytes(p));
+  const size_t tb = p->attn_path == 1 ? 0 : round256(blk_bytes(p)), cb = round256(cent_bytes(p));
   void* q_blk = w; w += tb;
   void* k_blk = w; w += tb;
   void* v_blk = w; w += tb;
@@ -390,6 +511,8 @@ bsa_status bsa_forward(bsa_plan_t p, const void* q, const void* k, const void* v
   if (idx_out) idx = idx_out;
   if (cnt_out) cnt = cnt_out;
   cudaStream_t st = (cudaStream_t)stream;
+  if (p->attn_path == 1)
+    return run_forward_fused(p, q, k, v, mode, param, kmax, o, idx, cnt, qc, kc, dev_status, st);
   if ((s = bsa_permute_qkv(p, q, k, v, q_blk, k_blk, v_blk, qc, kc, stream)) != BSA_OK) return s;
   if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st)) != BSA_OK) return s;
   if ((s = run_attention(p, q_blk, k_blk, v_blk, idx, cnt, kmax, o_blk, dev_status, st)) != BSA_OK) return s;

@@ -241,10 +241,40 @@ __device__ __forceinline__ bool for_each_event(int n0, int n1, F&& f) {
   return true;
 }
 
-template <int HD>
+// Issues the TMA loads of one 128-row tile (Q, K or V of block j of head
+// bh) into shared memory at dst, completing on bar.  Blocked layout: a 2D box
+// of the block's contiguous rows.  Original layout (ORIG): a 5D box
+// (d, head, x, y, t) whose shared-memory row order is the block's slot order
+// (dt, dy, dx) and whose out-of-range part (the grid's padding) is zero-filled,
+// or a 3D box (d, head, token) over the text tokens.
+template <bool ORIG, int HD>
+__device__ __forceinline__ void load_tile(const TileMaps& m, int which, const Geo& g, long long bh,
+                                          int j, uint32_t dst, uint32_t bar) {
+  constexpr int kPanel = 128 * 128;
+  if (!ORIG) {
+    const int row = (int)((bh * (g.nb + g.nb_text) + j) * 128);
+    const CUtensorMap* map = which == 0 ? &m.q : (which == 1 ? &m.k : &m.v);
+#pragma unroll
+    for (int p = 0; p < HD / 64; ++p) tma_load_2d(dst + p * kPanel, map, 64 * p, row, bar);
+  } else {
+    const int h = (int)(bh % g.Hd);
+    if (j < g.nb) {
+      const int xb = j % g.nbx, yb = (j / g.nbx) % g.nby, tb = j / (g.nbx * g.nby);
+      const CUtensorMap* map = which == 0 ? &m.q : (which == 1 ? &m.k : &m.v);
+#pragma unroll
+      for (int p = 0; p < HD / 64; ++p)
+        tma_load_5d(dst + p * kPanel, map, 64 * p, h, xb * g.bc, yb * g.br, tb * g.bf, bar);
+    } else {
+      const CUtensorMap* map = which == 0 ? &m.qt : (which == 1 ? &m.kt : &m.vt);
+#pragma unroll
+      for (int p = 0; p < HD / 64; ++p) tma_load_3d(dst + p * kPanel, map, 64 * p, h, (j - g.nb) * 128, bar);
+    }
+  }
+}
+
+template <int HD, bool ORIG>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    attn_tc_kernel(Geo g, AttnArgs a, const __grid_constant__ CUtensorMap tq,
-                   const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
+    attn_tc_kernel(Geo g, AttnArgs a, const __grid_constant__ TileMaps maps) {
   using L = TcLayout<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -307,10 +337,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       for (int x = 0; x < 2; ++x) {
         if ((x ? n1 : n0) == 0) continue;
-        const int qrow = (int)(((x ? bh1 : bh0) * nbk + (x ? i1 : i0)) * 128);
         mbar_arrive_expect_tx(bar(L::kBarQ + x), kTileBytes);
-        for (int p = 0; p < HD / 64; ++p)
-          tma_load_2d(sb + L::kQ + x * kTileBytes + p * L::kPanel, &tq, 64 * p, qrow, bar(L::kBarQ + x));
+        load_tile<ORIG, HD>(maps, 0, g, x ? bh1 : bh0, x ? i1 : i0, sb + L::kQ + x * kTileBytes,
+                            bar(L::kBarQ + x));
       }
       int pos = 0;
       bool bad = false;
@@ -321,11 +350,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (pos >= L::kStages &&
             !mbar_wait(bar(L::kBarEmpty + slot), ((pos / L::kStages) - 1) & 1, abort))
           return false;
-        const int row = (int)(((x ? bh1 : bh0) * nbk + j) * 128);
         const uint32_t dst = sRing + slot * kTileBytes;
         mbar_arrive_expect_tx(bar(L::kBarFull + slot), kTileBytes);
-        for (int p = 0; p < HD / 64; ++p)
-          tma_load_2d(dst + p * L::kPanel, kind == 0 ? &tk : &tv, 64 * p, row, bar(L::kBarFull + slot));
+        load_tile<ORIG, HD>(maps, kind == 0 ? 1 : 2, g, x ? bh1 : bh0, j, dst, bar(L::kBarFull + slot));
         ++pos;
         return true;
       });
@@ -487,10 +514,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       const uint4 qm = __ldg(reinterpret_cast<const uint4*>(a.masks) + qi);
       const uint32_t qw4[4] = {qm.x, qm.y, qm.z, qm.w};
-      const bool row_valid = ((qw4[r >> 5] >> (r & 31)) & 1u) && ok && n > 0;
+      const bool slot_real = (qw4[r >> 5] >> (r & 31)) & 1u;
+      const bool row_valid = slot_real && ok && n > 0;
       const float inv = (row_valid && l > 0.f) ? 1.f / l : 0.f;
-      uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) +
-                                             ((qbh * nbk + qi) * 128 + r) * HD);
+      // Blocked layout: every slot row is written (pad rows 0).  Original
+      // layout: each real slot's row goes to its token, pad slots are dropped.
+      long long orow_idx;
+      if (!ORIG) {
+        orow_idx = (qbh * nbk + qi) * 128 + r;
+      } else {
+        const long long tok = slot_token(g, qi, r);
+        orow_idx = tok >= 0 ? tok * g.Hd + (qbh % g.Hd) : -1;
+      }
+      uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + (orow_idx < 0 ? 0 : orow_idx) * HD);
 #pragma unroll
       for (int c0 = 0; c0 < HD; c0 += 32) {
         uint32_t orr[32];
@@ -508,7 +544,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           v.y = pack_bf16x2(__uint_as_float(orr[8 * c8 + 2]) * inv, __uint_as_float(orr[8 * c8 + 3]) * inv);
           v.z = pack_bf16x2(__uint_as_float(orr[8 * c8 + 4]) * inv, __uint_as_float(orr[8 * c8 + 5]) * inv);
           v.w = pack_bf16x2(__uint_as_float(orr[8 * c8 + 6]) * inv, __uint_as_float(orr[8 * c8 + 7]) * inv);
-          orow[c0 / 8 + c8] = v;
+          if (orow_idx >= 0) orow[c0 / 8 + c8] = v;
         }
       }
     }
@@ -527,30 +563,40 @@ size_t attn_tc_smem_bytes(int D) {
   return D == 128 ? TcLayout<128>::kAlloc : TcLayout<64>::kAlloc;
 }
 
-cudaError_t launch_attn_tc(const Geo& g, const AttnArgs& a, const CUtensorMap& tq,
-                           const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
-  const int tiles = g.B * g.Hd * (g.nb + g.nb_text);
-  if (tiles == 0) return cudaSuccess;
-  const int ctas = (tiles + 1) / 2;
+template <int HD, bool ORIG>
+static cudaError_t launch_tc_t(const Geo& g, const AttnArgs& a, const TileMaps& maps, int ctas,
+                               cudaStream_t st) {
   // The setmaxnreg split assumes the launch gives every thread exactly
   // kRegsLaunch registers; refuse to launch a build where that is not so.
   cudaFuncAttributes attr;
-  cudaError_t e = g.D == 128 ? cudaFuncGetAttributes(&attr, attn_tc_kernel<128>)
-                             : cudaFuncGetAttributes(&attr, attn_tc_kernel<64>);
+  cudaError_t e = cudaFuncGetAttributes(&attr, attn_tc_kernel<HD, ORIG>);
   if (e != cudaSuccess) return e;
   if (attr.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
-  if (g.D == 128) {
-    const int smem = TcLayout<128>::kAlloc;
-    e = cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attn_tc_kernel<128><<<ctas, kTcThreads, smem, st>>>(g, a, tq, tk, tv);
-  } else {
-    const int smem = TcLayout<64>::kAlloc;
-    e = cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attn_tc_kernel<64><<<ctas, kTcThreads, smem, st>>>(g, a, tq, tk, tv);
-  }
+  const int smem = TcLayout<HD>::kAlloc;
+  e = cudaFuncSetAttribute(attn_tc_kernel<HD, ORIG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  attn_tc_kernel<HD, ORIG><<<ctas, kTcThreads, smem, st>>>(g, a, maps);
   return cudaGetLastError();
+}
+
+// Blocked layout in and out (bsa_attention).
+cudaError_t launch_attn_tc(const Geo& g, const AttnArgs& a, const TileMaps& maps, cudaStream_t st) {
+  const int tiles = g.B * g.Hd * (g.nb + g.nb_text);
+  if (tiles == 0) return cudaSuccess;
+  const int ctas = (tiles + 1) / 2;
+  return g.D == 128 ? launch_tc_t<128, false>(g, a, maps, ctas, st)
+                    : launch_tc_t<64, false>(g, a, maps, ctas, st);
+}
+
+// Original layout in and out, one batch element (g.B == 1): the layout
+// transform and its inverse happen inside the loads and the epilogue.
+cudaError_t launch_attn_tc_orig(const Geo& g, const AttnArgs& a, const TileMaps& maps,
+                                cudaStream_t st) {
+  const int tiles = g.Hd * (g.nb + g.nb_text);
+  if (tiles == 0 || g.B != 1) return g.B != 1 ? cudaErrorInvalidValue : cudaSuccess;
+  const int ctas = (tiles + 1) / 2;
+  return g.D == 128 ? launch_tc_t<128, true>(g, a, maps, ctas, st)
+                    : launch_tc_t<64, true>(g, a, maps, ctas, st);
 }
 
 }  // namespace bsa

@@ -38,6 +38,13 @@ struct AttnArgs {
   float scale_log2;       // log2(e)/sqrt(D)
 };
 
+// TMA tensor maps of one attention launch: q/k/v cover the blocked tensors
+// (2D) or the video tokens of the original layout (5D); qt/kt/vt cover the
+// text tokens of the original layout (3D, unused otherwise).
+struct TileMaps {
+  CUtensorMap q, k, v, qt, kt, vt;
+};
+
 // permute.cu
 cudaError_t launch_permute(const Geo& g, bool is_bf16, const GatherArgs& a, cudaStream_t st);
 cudaError_t launch_unpermute(const Geo& g, bool is_bf16, const GatherArgs& a, cudaStream_t st);
@@ -48,7 +55,9 @@ cudaError_t launch_select(const Geo& g, const SelectArgs& a, cudaStream_t st);
 // attn.cu
 size_t attn_tc_smem_bytes(int D);
 cudaError_t launch_attn_simt(const Geo& g, bool is_bf16, const AttnArgs& a, cudaStream_t st);
-cudaError_t launch_attn_tc(const Geo& g, const AttnArgs& a, const CUtensorMap& tq,
-                           const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st);
+cudaError_t launch_attn_tc(const Geo& g, const AttnArgs& a, const TileMaps& maps, cudaStream_t st);
+cudaError_t launch_attn_tc_orig(const Geo& g, const AttnArgs& a, const TileMaps& maps,
+                                cudaStream_t st);
+cudaError_t launch_pool_orig(const Geo& g, bool is_bf16, const GatherArgs& a, cudaStream_t st);
 
 }  // namespace bsa

@@ -17,7 +17,7 @@
 
 namespace bsa {
 
-enum GatherMode { kPermute = 0, kUnpermute = 1, kPool = 2 };
+enum GatherMode { kPermute = 0, kUnpermute = 1, kPool = 2, kPoolOrig = 3 };
 
 
 constexpr int kGatherThreads = 256;
@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(Geo g, GatherArg
       tok[u] = s < g.bs ? s_tok[s] : -2;
       buf[u] = make_uint4(0, 0, 0, 0);
       if (tok[u] >= 0) {
-        const long long vi = (MODE == kPermute)
+        const long long vi = (MODE == kPermute || MODE == kPoolOrig)
                                  ? ((tok_base + tok[u]) * g.Hd + h) * V + vec
                                  : (blk_row0 + s) * V + vec;
         buf[u] = __ldg(src + vi);
@@ -124,6 +124,14 @@ cudaError_t launch_unpermute(const Geo& g, bool is_bf16, const GatherArgs& a, cu
   const int nblocks = g.nb + g.nb_text;
   return is_bf16 ? launch_gather_t<__nv_bfloat16, kUnpermute>(g, a, nblocks, st)
                  : launch_gather_t<float, kUnpermute>(g, a, nblocks, st);
+}
+
+// Centroids of the video blocks straight from the original layout (the
+// summarizer pass of the fused forward, which never materialises the blocked
+// tensors).
+cudaError_t launch_pool_orig(const Geo& g, bool is_bf16, const GatherArgs& a, cudaStream_t st) {
+  return is_bf16 ? launch_gather_t<__nv_bfloat16, kPoolOrig>(g, a, g.nb, st)
+                 : launch_gather_t<float, kPoolOrig>(g, a, g.nb, st);
 }
 
 // Centroids of the video blocks straight from the blocked layout.

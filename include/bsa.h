@@ -138,6 +138,14 @@ bsa_status bsa_permute_qkv(bsa_plan_t plan, const void* q, const void* k,
                            void* v_blk, float* q_cent, float* k_cent,
                            void* stream);
 
+/* bsa_centroids — the mean summarizer straight from the original layout
+ * (SPADE §3.1 MEAN-SPADE (q_mean, k_mean); §3.3 summaries Q', K'), without
+ * materialising the blocked tensors: the same values bsa_permute writes.
+ *   q, k            [B, Ntot, Hd, D] original order (read only)
+ *   q_cent, k_cent  [B, Hd, nb, D] float out (either may be NULL). */
+bsa_status bsa_centroids(bsa_plan_t plan, const void* q, const void* k,
+                         float* q_cent, float* k_cent, void* stream);
+
 /* bsa_unpermute — restore blocked output to the original token order (SPADE
  * §3.3, "output blocks are restored to the original layout"); pad slots are
  * dropped.   o_blk [B, Hd, Npad_tot, D] -> o [B, Ntot, Hd, D]. */
@@ -211,8 +219,26 @@ bsa_status bsa_attention(bsa_plan_t plan, const void* q_blk, const void* k_blk,
                          const int32_t* cnt, int kmax, void* o_blk,
                          int32_t* dev_status, void* stream);
 
-/* bsa_forward — the whole executor on one stream: permute (+centroids) ->
- * select -> attention -> unpermute (SPADE §3.3, Fig. 2(c)).
+/* bsa_attention_orig — bsa_attention on the ORIGINAL layout: the layout
+ * transform is fused into the tile loads (a 5D TMA box (d, head, x, y, t) per
+ * block, out-of-grid elements read as 0; a 3D box for text blocks) and its
+ * inverse into the epilogue (each real slot's row is written to its token).
+ * SPADE §3.3 "(1) Operator fusion ... (2) fuse Q/K gather-scatter with the
+ * layout transform".
+ *   q, k, v   [B, Ntot, Hd, D] original order;  o  [B, Ntot, Hd, D] out
+ *   idx, cnt, kmax, dev_status  as for bsa_attention
+ * Tensor-core plans only (bf16, 128-token blocks): other plans get
+ * BSA_ERR_UNSUPPORTED. */
+bsa_status bsa_attention_orig(bsa_plan_t plan, const void* q, const void* k,
+                              const void* v, const int32_t* idx,
+                              const int32_t* cnt, int kmax, void* o,
+                              int32_t* dev_status, void* stream);
+
+/* bsa_forward — the whole executor on one stream (SPADE §3.3, Fig. 2(c)).
+ * Tensor-core plans: bsa_centroids -> selection -> bsa_attention_orig (the
+ * layout transform and its inverse are fused into the attention's loads and
+ * stores).  Other plans: permute (+centroids) -> selection -> attention ->
+ * unpermute through blocked workspace tensors.
  *   q, k, v, o        original-order tensors [B, Ntot, Hd, D]
  *   idx_out, cnt_out  optional copies of the lists (NULL = keep internal)
  *   kmax              list width (>= bsa_kmax_for result)

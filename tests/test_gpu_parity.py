@@ -108,6 +108,49 @@ def test_attention_and_forward(name, dev):
     check_output(to_np(out), ref, w.dtype, f"{name} forward")
 
 
+@pytest.mark.parametrize("name", list(SMALL))
+def test_centroids_from_original_layout(name, dev):
+    w = SMALL[name]
+    g = geometry(w)
+    (q, k, _), (qd, kd, _) = _inputs(w, dev)
+    plan = bsa.plan_for(w, dev)
+    qc, kc = plan.centroids(qd, kd)
+    _, qc_perm = plan.permute(qd, centroids=True)
+    torch.cuda.synchronize()
+    # same fixed summation order as the fused permute: identical values
+    assert torch.equal(qc, qc_perm)
+    np.testing.assert_allclose(kc.cpu().numpy(), orc.centroids(g, to_np(k)), rtol=1e-5, atol=1e-5)
+
+
+@pytest.mark.parametrize("name", [n for n in SMALL if SMALL[n].dtype == "bf16" and SMALL[n].bs == 128])
+def test_attention_on_original_layout(name, dev):
+    w = SMALL[name]
+    g = geometry(w)
+    (q, k, v), (qd, kd, vd) = _inputs(w, dev)
+    plan = bsa.plan_for(w, dev)
+    qc, kc = plan.centroids(qd, kd)
+    idx, cnt = plan.select_centroids(qc, kc, w.mode, w.params)
+    out = plan.attention_orig(qd, kd, vd, idx, cnt)
+    qb, kb, vb, _, _ = plan.permute_qkv(qd, kd, vd)
+    blocked = plan.unpermute(plan.attention(qb, kb, vb, idx, cnt))
+    plan.check_status()
+    ref = orc.attention(g, to_np(q), to_np(k), to_np(v), idx.cpu().numpy(), cnt.cpu().numpy())
+    check_output(to_np(out), ref, w.dtype, f"{name} original layout")
+    # the fused layout transform reproduces the blocked path bit for bit
+    assert torch.equal(out, blocked)
+
+
+def test_attention_on_original_layout_needs_tensor_core_plan(dev):
+    w = SMALL["simt_bf16_bs32"]
+    (_, _, _), (qd, kd, vd) = _inputs(w, dev)
+    plan = bsa.plan_for(w, dev)
+    qc, kc = plan.centroids(qd, kd)
+    idx, cnt = plan.select_centroids(qc, kc, w.mode, w.params)
+    with pytest.raises(bsa.BsaError) as e:
+        plan.attention_orig(qd, kd, vd, idx, cnt)
+    assert e.value.status == 2
+
+
 def test_ones_values_give_ones(dev):
     w = SMALL["hy_ragged_text"]
     (_, _, _), (qd, kd, vd) = _inputs(w, dev)
