@@ -65,6 +65,24 @@ __device__ int count_at_least(const float* row, int nb, uint32_t cand, int lane)
   return c;
 }
 
+// Lanes hold the order keys of their scores (j = lane + 32 e) in registers,
+// so the 32-step threshold search does not re-read shared memory.
+constexpr int kKeysPerLane = 48;   // register-resident search for nb <= 1536
+
+// Largest T with #{j : key_j >= T} >= k (the k-th largest key), bit by bit.
+__device__ __forceinline__ uint32_t kth_largest_key(const uint32_t (&kr)[kKeysPerLane], int k) {
+  uint32_t T = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    int c = 0;
+#pragma unroll
+    for (int e = 0; e < kKeysPerLane; ++e) c += kr[e] >= cand ? 1 : 0;   // pad keys are 0
+    c = __reduce_add_sync(0xffffffffu, c);
+    if (c >= k) T = cand;
+  }
+  return T;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, SelectArgs a) {
   extern __shared__ __align__(16) float sm[];
@@ -122,7 +140,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, SelectArgs a
     for (int j = lane; j < nb; j += 32) m = fmaxf(m, row[j]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    const double Z = mass_at_least(row, nb, m, 0u, lane);
+    // The normaliser is needed only for the score output and for Top-P
+    // (Top-K depends on the order of the scores alone).
+    const double Z = (a.scores != nullptr || a.mode != 0) ? mass_at_least(row, nb, m, 0u, lane) : 1.0;
 
     if (a.scores != nullptr) {
       float* out = a.scores + (bh * nb + i) * nb;
@@ -133,12 +153,28 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, SelectArgs a
     int need = 0;  // how many of the scores equal to the threshold to take
     if (a.mode == 0) {
       const int k = (int)a.param[h];
-      for (int bit = 31; bit >= 0; --bit) {
-        const uint32_t cand = T | (1u << bit);
-        if (count_at_least(row, nb, cand, lane) >= k) T = cand;
+      if (nb <= 32 * kKeysPerLane) {
+        // order_key of any float is nonzero and every candidate threshold is
+        // nonzero, so the 0 used for missing entries never counts
+        uint32_t kr[kKeysPerLane];
+#pragma unroll
+        for (int e = 0; e < kKeysPerLane; ++e) {
+          const int j = lane + 32 * e;
+          kr[e] = j < nb ? order_key(row[j]) : 0u;
+        }
+        T = kth_largest_key(kr, k);
+        int c = 0;
+#pragma unroll
+        for (int e = 0; e < kKeysPerLane; ++e) c += kr[e] > T ? 1 : 0;
+        need = k - __reduce_add_sync(0xffffffffu, c);
+      } else {
+        for (int bit = 31; bit >= 0; --bit) {
+          const uint32_t cand = T | (1u << bit);
+          if (count_at_least(row, nb, cand, lane) >= k) T = cand;
+        }
+        const int n_gt = (T == 0xffffffffu) ? 0 : count_at_least(row, nb, T + 1, lane);
+        need = k - n_gt;
       }
-      const int n_gt = (T == 0xffffffffu) ? 0 : count_at_least(row, nb, T + 1, lane);
-      need = k - n_gt;
     } else {
       const double target = a.param[h] * Z;
       for (int bit = 31; bit >= 0; --bit) {
