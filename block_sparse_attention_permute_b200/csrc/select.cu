@@ -23,12 +23,13 @@ namespace bsa {
 
 
 constexpr int kSelRows = 16;      // query-block rows per CTA
-constexpr int kSelKeys = 64;      // key blocks per score chunk
+constexpr int kSelKeys = 256;     // key blocks per score chunk
+constexpr int kSelDChunk = 32;    // head-dim slice of a key chunk held in shared memory
 constexpr int kSelThreads = 256;  // 8 warps
 
 size_t select_smem_bytes(int nb, int D) {
-  return sizeof(float) *
-         ((size_t)kSelRows * D + (size_t)kSelKeys * (D + 4) + (size_t)kSelRows * nb);
+  return sizeof(float) * ((size_t)kSelRows * D + (size_t)kSelKeys * (kSelDChunk + 4) +
+                          (size_t)kSelRows * nb);
 }
 
 __device__ __forceinline__ uint32_t order_key(float s) {
@@ -87,8 +88,8 @@ template <int D>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, SelectArgs a) {
   extern __shared__ __align__(16) float sm[];
   float* qs = sm;                                   // [kSelRows][D]
-  float* ks = qs + kSelRows * D;                    // [kSelKeys][D+4]
-  float* sc = ks + kSelKeys * (D + 4);              // [kSelRows][nb]
+  float* ks = qs + kSelRows * D;                    // [kSelKeys][kSelDChunk+4]
+  float* sc = ks + kSelKeys * (kSelDChunk + 4);     // [kSelRows][nb]
   const int nb = g.nb;
   const int h = blockIdx.y, b = blockIdx.z;
   const long long bh = (long long)b * g.Hd + h;
@@ -96,37 +97,52 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, SelectArgs a
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   // ---- phase 1: scores of kSelRows query blocks against all key blocks ----
+  // Thread (ty, tx) accumulates rows 8ty..8ty+7 against keys tx and tx+128 of
+  // each 256-key chunk; the chunk's keys pass through shared memory 32
+  // dimensions at a time.  Each dot product is one fma chain over d in
+  // ascending order, the same as a plain sequential loop.
   for (int e = tid; e < kSelRows * D; e += kSelThreads) {
     const int r = e / D, d = e % D;
     qs[e] = (i0 + r < nb) ? a.qc[(bh * nb + i0 + r) * D + d] : 0.f;
   }
-  const int tx = tid % kSelKeys;     // key within chunk
-  const int ty = tid / kSelKeys;     // row group: rows 4*ty .. 4*ty+3
+  const int ty = tid / 128, tx = tid % 128;
+  constexpr int KS = kSelDChunk + 4;               // padded row: conflict-free float4 reads
   for (int j0 = 0; j0 < nb; j0 += kSelKeys) {
-    __syncthreads();
-    for (int e = tid; e < kSelKeys * (D / 4); e += kSelThreads) {
-      const int jj = e / (D / 4), d4 = e % (D / 4);
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j0 + jj < nb) v = *reinterpret_cast<const float4*>(a.kc + (bh * nb + j0 + jj) * D + 4 * d4);
-      *reinterpret_cast<float4*>(ks + jj * (D + 4) + 4 * d4) = v;
-    }
-    __syncthreads();
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int d4 = 0; d4 < D / 4; ++d4) {
-      const float4 kv = *reinterpret_cast<const float4*>(ks + tx * (D + 4) + 4 * d4);
+    float acc[8][2];
 #pragma unroll
-      for (int rr = 0; rr < 4; ++rr) {
-        const float4 qv = *reinterpret_cast<const float4*>(qs + (4 * ty + rr) * D + 4 * d4);
-        acc[rr] = fmaf(qv.x, kv.x, acc[rr]);
-        acc[rr] = fmaf(qv.y, kv.y, acc[rr]);
-        acc[rr] = fmaf(qv.z, kv.z, acc[rr]);
-        acc[rr] = fmaf(qv.w, kv.w, acc[rr]);
+    for (int r = 0; r < 8; ++r) acc[r][0] = acc[r][1] = 0.f;
+    for (int d0 = 0; d0 < D; d0 += kSelDChunk) {
+      __syncthreads();
+      for (int e = tid; e < kSelKeys * (kSelDChunk / 4); e += kSelThreads) {
+        const int jj = e / (kSelDChunk / 4), d4 = e % (kSelDChunk / 4);
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (j0 + jj < nb)
+          v = *reinterpret_cast<const float4*>(a.kc + (bh * nb + j0 + jj) * D + d0 + 4 * d4);
+        *reinterpret_cast<float4*>(ks + jj * KS + 4 * d4) = v;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int d4 = 0; d4 < kSelDChunk / 4; ++d4) {
+        const float4 k0 = *reinterpret_cast<const float4*>(ks + tx * KS + 4 * d4);
+        const float4 k1 = *reinterpret_cast<const float4*>(ks + (tx + 128) * KS + 4 * d4);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const float4 qv = *reinterpret_cast<const float4*>(qs + (8 * ty + r) * D + d0 + 4 * d4);
+          acc[r][0] = fmaf(qv.x, k0.x, acc[r][0]);
+          acc[r][0] = fmaf(qv.y, k0.y, acc[r][0]);
+          acc[r][0] = fmaf(qv.z, k0.z, acc[r][0]);
+          acc[r][0] = fmaf(qv.w, k0.w, acc[r][0]);
+          acc[r][1] = fmaf(qv.x, k1.x, acc[r][1]);
+          acc[r][1] = fmaf(qv.y, k1.y, acc[r][1]);
+          acc[r][1] = fmaf(qv.z, k1.z, acc[r][1]);
+          acc[r][1] = fmaf(qv.w, k1.w, acc[r][1]);
+        }
       }
     }
-    if (j0 + tx < nb) {
 #pragma unroll
-      for (int rr = 0; rr < 4; ++rr) sc[(4 * ty + rr) * nb + j0 + tx] = acc[rr] * a.scale + 0.0f;
+    for (int r = 0; r < 8; ++r) {
+      if (j0 + tx < nb) sc[(8 * ty + r) * nb + j0 + tx] = acc[r][0] * a.scale + 0.0f;
+      if (j0 + tx + 128 < nb) sc[(8 * ty + r) * nb + j0 + tx + 128] = acc[r][1] * a.scale + 0.0f;
     }
   }
   __syncthreads();
