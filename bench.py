@@ -90,7 +90,7 @@ def profiled_traffic(workload: str):
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled during the timed region."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -102,11 +102,19 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.5)            # let the sampler start before the timed region
         except (FileNotFoundError, OSError):
             self.proc = None
+        self.t_start = self.t_end = None
         return self
+
+    def mark_start(self):
+        self.t_start = time.time()
+
+    def mark_end(self):
+        self.t_end = time.time()
 
     def __exit__(self, *exc):
         self.lines = []
@@ -120,18 +128,25 @@ class ClockSampler:
             self.lines = [ln for ln in out.splitlines() if ln.strip()]
 
     def summary(self):
+        """Median SM clock and throttle reasons over the samples taken inside the
+        timed region (timestamps between mark_start and mark_end)."""
+        from datetime import datetime
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in getattr(self, "lines", []):
             parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                ts = datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                clk, clk_max = float(parts[2]), float(parts[3])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+            if self.t_start is not None and not (self.t_start <= ts <= (self.t_end or ts)):
+                continue
+            sm.append(clk)
+            mx = clk_max
+            for n, v in zip(names, parts[6:10]):
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
@@ -226,11 +241,13 @@ def run_ours(args, rank, world, local):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     with ClockSampler(local) as clk:
+        clk.mark_start()
         ev0.record(stream)
         for _ in range(args.steps):
             forward()
         ev1.record(stream)
         barrier()
+        clk.mark_end()
     plan.check_status()
     step_ms = ev0.elapsed_time(ev1) / args.steps
     clocks = clk.summary()
@@ -277,27 +294,75 @@ def run_ours(args, rank, world, local):
     del qb, kb, vb, ob
     phase_ms = fused if fused is not None else unfused
 
-    # ---- end to end: pinned host buffers, copies inside the timed region
+    # ---- end to end: pinned host buffers, copies inside the timed region.
+    # Serial: upload, forward, download on one stream.  Pipelined: three
+    # streams and double-buffered device tensors, so step i+1's upload runs
+    # while step i computes and step i-1's output downloads; every step still
+    # moves its own inputs up and its own output down.
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
-    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    ohs = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(2)]
+    h2d = 3 * q.numel() * q.element_size()
+    d2h = q.numel() * q.element_size()
+
+    def upload(dst):
+        for d_t, h_t in zip(dst, (qh, kh, vh)):
+            d_t.copy_(h_t, non_blocking=True)
+
     for _ in range(2):
-        qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
-        forward()
-        oh.copy_(out, non_blocking=True)
+        upload((qd, kd, vd)); forward(); ohs[0].copy_(out, non_blocking=True)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
-        forward()
-        oh.copy_(out, non_blocking=True)
+        upload((qd, kd, vd)); forward(); ohs[0].copy_(out, non_blocking=True)
     e1.record(stream)
     barrier()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    h2d = 3 * q.numel() * q.element_size()
-    d2h = q.numel() * q.element_size()
+    e2e_serial_ms = e0.elapsed_time(e1) / args.steps
+    ref_out = ohs[0].clone()
 
-    step_ms, e2e_ms, attn_ms = reduce_max([step_ms, e2e_ms, phase_ms["attention"]], dev)
+    ins = [(qd, kd, vd), tuple(torch.empty_like(t) for t in (qd, kd, vd))]
+    outs = [out, torch.empty_like(out)]
+    s_up, s_dn = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_dn = [torch.cuda.Event() for _ in range(2)]
+
+    def run_pipelined(n_steps, first_event=None):
+        for i in range(n_steps):
+            bi = i % 2
+            with torch.cuda.stream(s_up):
+                if i >= 2:
+                    s_up.wait_event(ev_done[bi])            # compute i-2 finished reading ins[bi]
+                if i == 0 and first_event is not None:
+                    first_event.record(s_up)
+                upload(ins[bi])
+                ev_in[bi].record(s_up)
+            stream.wait_event(ev_in[bi])
+            if i >= 2:
+                stream.wait_event(ev_dn[bi])                 # download i-2 finished reading outs[bi]
+            qi, ki, vi = ins[bi]
+            bsa._check(L.bsa_forward(plan._h, P(qi), P(ki), P(vi), w.mode, params, kmax,
+                                     P(outs[bi]), P(idx), P(cnt), P(ws), ws.numel(), None,
+                                     bsa._stream(dev)))
+            ev_done[bi].record(stream)
+            with torch.cuda.stream(s_dn):
+                s_dn.wait_event(ev_done[bi])
+                ohs[bi].copy_(outs[bi], non_blocking=True)
+                ev_dn[bi].record(s_dn)
+
+    run_pipelined(3)
+    barrier()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    run_pipelined(args.steps, first_event=p0)
+    p1.record(s_dn)
+    barrier()
+    e2e_ms = p0.elapsed_time(p1) / args.steps
+    # the overlapped steps did all their work: the last downloaded output equals
+    # the serial loop's (same inputs, deterministic kernels)
+    assert torch.equal(ohs[(args.steps - 1) % 2], ref_out), "pipelined e2e output differs"
+
+    step_ms, e2e_ms, e2e_serial_ms, attn_ms = reduce_max(
+        [step_ms, e2e_ms, e2e_serial_ms, phase_ms["attention"]], dev)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -353,7 +418,11 @@ def run_ours(args, rank, world, local):
         },
         "e2e": {"value": round(job_tflops(world, flops, e2e_ms), 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h,
+                "mode": "pipelined across steps (upload / compute / download streams, "
+                        "double-buffered device tensors)",
+                "serial": {"value": round(job_tflops(world, flops, e2e_serial_ms), 2),
+                           "ms_per_step": round(e2e_serial_ms, 3)}},
         "gpu_launches": (3 if plan.info.attn_path == 1 else 4) * args.steps,
         "clocks": clocks,
     }
@@ -440,8 +509,8 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="hunyuan", choices=synthetic.WORKLOADS)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
