@@ -53,6 +53,9 @@ def _load():
         lib.orc_k_for_density.restype = ctypes.c_int
         lib.orc_select.argtypes = [P, P, ctypes.c_int, P, ctypes.c_int, P, P, P]
         lib.orc_attention.argtypes = [P, P, P, P, P, P, ctypes.c_int, P, ctypes.c_longlong, P]
+        lib.orc_sics.argtypes = [P, P, P]
+        lib.orc_sics_online.argtypes = [P, P, P]
+        lib.orc_aggregation_score.argtypes = [P, P, P]
         lib.orc_selected_pairs.argtypes = [P, P, P, ctypes.c_int]
         lib.orc_selected_pairs.restype = ctypes.c_longlong
         _lib = lib
@@ -169,6 +172,37 @@ def attention(g: Geometry, q, k, v, idx, cnt, rows=None):
         _load().orc_attention(_ptr(g.arr), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt),
                               kmax, _ptr(rows), len(rows), _ptr(out))
     return out
+
+
+def sics(g: Geometry, x):
+    """Sum of intra-block cosine similarities per video block, [B,Hd,nb] (SPADE Eq. (4))."""
+    x = _f32(x)
+    out = np.empty((g.B, g.Hd, g.nb), dtype=np.float64)
+    _load().orc_sics(_ptr(g.arr), _ptr(x), _ptr(out))
+    return out
+
+
+def sics_online(g: Geometry, x):
+    """The same by the online form (SPADE Eq. (5), Algorithm 1), [B,Hd,nb]."""
+    x = _f32(x)
+    out = np.empty((g.B, g.Hd, g.nb), dtype=np.float64)
+    _load().orc_sics_online(_ptr(g.arr), _ptr(x), _ptr(out))
+    return out
+
+
+def aggregation_score(g: Geometry, x):
+    """AS = sum of SICS over video blocks, [B,Hd] (SPADE Eq. (3))."""
+    x = _f32(x)
+    out = np.empty((g.B, g.Hd), dtype=np.float64)
+    _load().orc_aggregation_score(_ptr(g.arr), _ptr(x), _ptr(out))
+    return out
+
+
+def choose_scheme(geoms, x):
+    """Per (b, h): index of the candidate geometry (blocking scheme) with the largest AS,
+    lowest index on equality (SPADE §3.2: the Selected Blocking Scheme has max AS)."""
+    scores = np.stack([aggregation_score(g, x) for g in geoms])   # [n, B, Hd]
+    return np.argmax(scores, axis=0).astype(np.int32), scores
 
 
 def selected_pairs(g: Geometry, idx, cnt) -> int:

@@ -36,6 +36,7 @@
 //   R8 text blocks are not scored; every video query block also attends all
 //      text key blocks; text query tokens attend every token.
 //   R9 lists are stored in ascending block id, text blocks last.
+//   R15 SICS: a zero vector has no direction and contributes nothing.
 //
 // Geometry array g[10] = {B, T, H, W, bf, br, bc, Hd, D, n_text}.
 
@@ -342,6 +343,79 @@ void orc_attention(const int* g, const float* q, const float* k, const float* v,
       for (long long d = 0; d < G.D; ++d) out[d] += w * (double)vv[d];
     }
   });
+}
+
+// Intra-block estimator (SPADE §3.2, Eq. (4)): the sum over all ordered pairs
+// (a, b) of valid tokens of a block of the cosine similarity
+// q_a.q_b / (|q_a| |q_b|), diagonal included.  Reading R15: a zero vector has
+// no direction and contributes nothing.  x [B, Ntot, Hd, D] -> out [B, Hd, nb].
+void orc_sics(const int* g, const float* x, double* out) {
+  Geom G = make_geom(g);
+  parallel_for(G.B * G.Hd * G.nb, [&](long long task) {
+    long long b = task / (G.Hd * G.nb), h = (task / G.nb) % G.Hd, j = task % G.nb;
+    std::vector<long long> toks = block_tokens(G, j);
+    std::vector<double> u(toks.size() * G.D, 0.0);
+    for (size_t a = 0; a < toks.size(); ++a) {
+      const float* v = x + ((b * G.n_tot + toks[a]) * G.Hd + h) * G.D;
+      double nrm = 0.0;
+      for (long long d = 0; d < G.D; ++d) nrm += (double)v[d] * (double)v[d];
+      nrm = std::sqrt(nrm);
+      if (nrm > 0.0)
+        for (long long d = 0; d < G.D; ++d) u[a * G.D + d] = (double)v[d] / nrm;
+    }
+    double s = 0.0;
+    for (size_t a = 0; a < toks.size(); ++a)
+      for (size_t c = 0; c < toks.size(); ++c) {
+        double dot = 0.0;
+        for (long long d = 0; d < G.D; ++d) dot += u[a * G.D + d] * u[c * G.D + d];
+        s += dot;
+      }
+    out[task] = s;
+  });
+}
+
+// The same quantity by the online form of SPADE §3.2 (Eq. (5), Algorithm 1):
+// walk the block's vectors in slot order, keeping the running sum r of the
+// normalised vectors seen so far and sigma += <r, qhat_j> before adding
+// qhat_j; the result is 2*sigma + (number of nonzero vectors).
+void orc_sics_online(const int* g, const float* x, double* out) {
+  Geom G = make_geom(g);
+  parallel_for(G.B * G.Hd * G.nb, [&](long long task) {
+    long long b = task / (G.Hd * G.nb), h = (task / G.nb) % G.Hd, j = task % G.nb;
+    std::vector<long long> toks = block_tokens(G, j);
+    std::vector<double> r(G.D, 0.0), qh(G.D);
+    double sigma = 0.0;
+    long long n = 0;
+    for (long long t : toks) {
+      const float* v = x + ((b * G.n_tot + t) * G.Hd + h) * G.D;
+      double nrm = 0.0;
+      for (long long d = 0; d < G.D; ++d) nrm += (double)v[d] * (double)v[d];
+      nrm = std::sqrt(nrm);
+      if (nrm == 0.0) continue;
+      double dot = 0.0;
+      for (long long d = 0; d < G.D; ++d) {
+        qh[d] = (double)v[d] / nrm;
+        dot += r[d] * qh[d];
+      }
+      sigma += dot;
+      for (long long d = 0; d < G.D; ++d) r[d] += qh[d];
+      ++n;
+    }
+    out[task] = 2.0 * sigma + (double)n;
+  });
+}
+
+// Aggregation score (SPADE §3.2, Eq. (3)): AS = sum over the video blocks of
+// SICS, per batch element and head.  as [B, Hd].
+void orc_aggregation_score(const int* g, const float* x, double* as) {
+  Geom G = make_geom(g);
+  std::vector<double> sics(G.B * G.Hd * G.nb);
+  orc_sics(g, x, sics.data());
+  for (long long bh = 0; bh < G.B * G.Hd; ++bh) {
+    double s = 0.0;
+    for (long long j = 0; j < G.nb; ++j) s += sics[bh * G.nb + j];
+    as[bh] = s;
+  }
 }
 
 // Number of (query token, key token) pairs the lists select, valid tokens

@@ -284,3 +284,53 @@ def test_selected_pairs_counts_mask_entries():
     g = orc.Geometry(**RAGGED)
     idx, cnt = random_lists(g, 28)
     assert orc.selected_pairs(g, idx, cnt) == int(token_mask(g, idx, cnt).sum())
+
+
+# ---------------------------------------------------------- SICS pins (SPADE §3.2)
+def test_sics_equals_squared_norm_of_summed_unit_vectors():
+    # Eq. (4) sums all pairwise cosines = || sum_k q_k/|q_k| ||^2 (algebra on Eq. (4))
+    g = orc.Geometry(**RAGGED)
+    x = rand_x(g, 40)
+    tab = token_table(g)
+    expect = np.zeros((g.B, g.Hd, g.nb))
+    for b in range(g.B):
+        for h in range(g.Hd):
+            for j in range(g.nb):
+                toks = tab[j][tab[j] >= 0]
+                v = x[b, toks, h, :].astype(np.float64)
+                u = v / np.linalg.norm(v, axis=1, keepdims=True)
+                expect[b, h, j] = np.sum(u.sum(0) ** 2)
+    np.testing.assert_allclose(orc.sics(g, x), expect, rtol=1e-12, atol=1e-10)
+
+
+def test_sics_online_algorithm_equals_definition():
+    g = orc.Geometry(**dict(RAGGED, D=24))
+    x = rand_x(g, 41)
+    np.testing.assert_allclose(orc.sics_online(g, x), orc.sics(g, x), rtol=1e-12, atol=1e-10)
+
+
+def test_sics_special_cases():
+    # identical directions -> every cosine is 1 -> n^2; mutually orthogonal -> n (the diagonal)
+    g = orc.Geometry(B=1, T=1, H=2, W=4, bf=1, br=2, bc=4, Hd=2, D=16, n_text=0)   # one block of 8
+    x = np.zeros((1, g.n_tot, 2, 16), dtype=np.float32)
+    x[0, :, 0, :] = np.arange(1, 17, dtype=np.float32) * 0.5          # head 0: all the same vector
+    x[0, :, 0, :] *= np.arange(1, 9, dtype=np.float32)[:, None]       # ... with different norms
+    x[0, :, 1, :] = np.eye(16, dtype=np.float32)[:8] * 3.0             # head 1: orthogonal
+    s = orc.sics(g, x)
+    assert abs(s[0, 0, 0] - 64.0) < 1e-9 and abs(s[0, 1, 0] - 8.0) < 1e-12
+    # a zero vector contributes nothing (reading R15)
+    x[0, 3, 1, :] = 0.0
+    assert abs(orc.sics(g, x)[0, 1, 0] - 7.0) < 1e-12
+    assert abs(orc.sics_online(g, x)[0, 1, 0] - 7.0) < 1e-12
+
+
+def test_aggregation_score_and_scheme_choice():
+    # AS = sum of block SICS (Eq. (3)); the chosen scheme maximises it
+    base = dict(B=1, T=4, H=8, W=8, Hd=3, D=16, n_text=0)
+    geoms = [orc.Geometry(bf=1, br=8, bc=8, **base), orc.Geometry(bf=4, br=4, bc=4, **base),
+             orc.Geometry(bf=2, br=2, bc=16, **base)]
+    x = rand_x(geoms[0], 42)
+    choice, scores = orc.choose_scheme(geoms, x)
+    for gi, g in enumerate(geoms):
+        np.testing.assert_allclose(scores[gi], orc.sics(g, x).sum(-1), rtol=1e-13)
+    assert np.all(scores[choice[0], 0, np.arange(3)] >= scores.max(0)[0] - 1e-12)
