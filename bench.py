@@ -23,6 +23,7 @@ sample of the same workload (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -191,6 +192,54 @@ def effective_pairs(plan, idx, cnt) -> int:
     return video + text
 
 
+CANDIDATE_SHAPES = [(1, 8, 16), (4, 4, 8), (16, 1, 8), (2, 8, 8), (8, 2, 8)]
+
+
+def time_scheme_generation(bsa, w, qd, dev, args, barrier):
+    """CUDA-event timing of bsa_aggregation_scores over three candidate block
+    shapes (the workload's own first), inputs resident (larger than L2)."""
+    shapes = [(w.bf, w.br, w.bc)] + [s for s in CANDIDATE_SHAPES if s != (w.bf, w.br, w.bc)][:2]
+    plans = [bsa.Plan(w.B, w.T, w.H, w.W, bf, br, bc, w.Hd, w.D, w.n_text, qd.dtype, dev)
+             for bf, br, bc in shapes]
+    L = bsa.load()
+    n = len(plans)
+    sics = [torch.empty((w.B, w.Hd, p.info.nb), dtype=torch.float32, device=dev) for p in plans]
+    as_ = torch.empty((n, w.B, w.Hd), dtype=torch.float64, device=dev)
+    choice = torch.empty((w.B, w.Hd), dtype=torch.int32, device=dev)
+    handles = (ctypes.c_void_p * n)(*[p._h.value for p in plans])
+    outs = (ctypes.c_void_p * n)(*[t.data_ptr() for t in sics])
+    stream = torch.cuda.current_stream(dev)
+
+    def call():
+        bsa._check(L.bsa_aggregation_scores(handles, n, bsa._ptr(qd), outs, bsa._ptr(as_),
+                                            bsa._ptr(choice), bsa._stream(dev)))
+
+    for _ in range(args.warmup):
+        call()
+    barrier()
+    # replayed from a CUDA graph of 10 calls, so host launch gaps do not count
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(10):
+            call()
+    graph.replay()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(1, args.steps // 10)
+    e0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    e1.record(stream)
+    barrier()
+    ms = e0.elapsed_time(e1) / (10 * reps)
+    del graph
+    x_bytes = qd.numel() * qd.element_size()
+    return {"candidates": [f"{a}x{b}x{c}" for a, b, c in shapes], "ms": round(ms, 4),
+            "algorithmic_bytes": x_bytes,
+            "achieved_gbs": round(x_bytes / (ms * 1e-3) / 1e9, 1),
+            "choice_histogram": torch.bincount(choice.flatten().long(), minlength=n).tolist()}
+
+
 def run_ours(args, rank, world, local):
     import block_sparse_attention_permute_b200 as bsa
 
@@ -293,6 +342,10 @@ def run_ours(args, rank, world, local):
          lambda: L.bsa_unpermute(plan._h, P(ob), P(out), S())])
     del qb, kb, vb, ob
     phase_ms = fused if fused is not None else unfused
+
+    # ---- scheme generation (aggregation evaluation over candidate blockings):
+    # one launch evaluates three candidate schemes of Q; timed alone.
+    scheme = time_scheme_generation(bsa, w, qd, dev, args, barrier)
 
     # ---- end to end: pinned host buffers, copies inside the timed region.
     # Serial: upload, forward, download on one stream.  Pipelined: three
@@ -423,6 +476,9 @@ def run_ours(args, rank, world, local):
                         "double-buffered device tensors)",
                 "serial": {"value": round(job_tflops(world, flops, e2e_serial_ms), 2),
                            "ms_per_step": round(e2e_serial_ms, 3)}},
+        "scheme_generation": dict(scheme, share_of_attn=round(scheme["ms"] / phase_ms["attention"], 4),
+                                  frac=round(scheme["achieved_gbs"] / hbm_gbs, 4),
+                                  peak_gbs=hbm_gbs, bound="hbm"),
         "gpu_launches": (3 if plan.info.attn_path == 1 else 4) * args.steps,
         "clocks": clocks,
     }

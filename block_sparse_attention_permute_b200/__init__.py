@@ -76,6 +76,8 @@ def load():
         "bsa_attention": [P, P, P, P, P, P, I, P, P, P],
         "bsa_forward": [P, P, P, P, I, P, I, P, P, P, P, Z, P, P],
         "bsa_check_status": [P, P],
+        "bsa_sics": [P, P, P, P],
+        "bsa_aggregation_scores": [P, I, P, P, P, P, P],
     }
     for name, args in sigs.items():
         fn = getattr(L, name)
@@ -201,6 +203,15 @@ class Plan:
                                     _stream(self.device)))
         return qc, kc
 
+    def sics(self, x, out=None):
+        """Sum of intra-block cosine similarities per video block, [B,Hd,nb] fp32 (bsa_sics)."""
+        self._check_tensor(x, self.orig_shape, name="x")
+        i = self.info
+        out = self._new((i.batch, i.heads, i.nb), torch.float32) if out is None else out
+        self._check_tensor(out, (i.batch, i.heads, i.nb), torch.float32, "out")
+        _check(load().bsa_sics(self._h, _ptr(x), _ptr(out), _stream(self.device)))
+        return out
+
     def attention_orig(self, q, k, v, idx, cnt, out=None, dev_status=None):
         """Attention on the original layout; the layout transform is fused (bsa_attention_orig)."""
         for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -280,6 +291,27 @@ class Plan:
     def check_status(self):
         """Synchronise the current stream and raise if a kernel recorded an error."""
         _check(load().bsa_check_status(self._h, _stream(self.device)))
+
+
+def aggregation_scores(plans, x):
+    """Aggregation evaluation over candidate blocking schemes (bsa_aggregation_scores).
+
+    plans: 1..8 Plans that differ only in block shape.  Returns (sics, as_, choice):
+    sics[c] [B,Hd,nb_c] fp32, as_ [n,B,Hd] float64, choice [B,Hd] int32.
+    """
+    plans = list(plans)
+    n = len(plans)
+    p0 = plans[0]
+    p0._check_tensor(x, p0.orig_shape, name="x")
+    i = p0.info
+    sics = [p._new((i.batch, i.heads, p.info.nb), torch.float32) for p in plans]
+    as_ = p0._new((n, i.batch, i.heads), torch.float64)
+    choice = p0._new((i.batch, i.heads), torch.int32)
+    handles = (ctypes.c_void_p * n)(*[p._h.value for p in plans])
+    outs = (ctypes.c_void_p * n)(*[t.data_ptr() for t in sics])
+    _check(load().bsa_aggregation_scores(handles, n, _ptr(x), outs, _ptr(as_), _ptr(choice),
+                                         _stream(p0.device)))
+    return sics, as_, choice
 
 
 def plan_for(w, device=None) -> Plan:

@@ -519,6 +519,46 @@ bsa_status bsa_forward(bsa_plan_t p, const void* q, const void* k, const void* v
   return bsa_unpermute(p, o_blk, o, stream);
 }
 
+bsa_status bsa_sics(bsa_plan_t p, const void* x, float* sics, void* stream) {
+  bsa_plan_t plans[1] = {p};
+  float* outs[1] = {sics};
+  return bsa_aggregation_scores(plans, 1, x, outs, nullptr, nullptr, stream);
+}
+
+bsa_status bsa_aggregation_scores(const bsa_plan_t* plans, int n_plans, const void* x,
+                                  float* const* sics, double* as, int32_t* choice, void* stream) {
+  if (plans == nullptr || sics == nullptr) return fail(BSA_ERR_INVALID_ARG, "NULL plan or SICS array");
+  if (n_plans < 1 || n_plans > bsa::kMaxSchemes)
+    return fail(BSA_ERR_INVALID_ARG, "n_plans = %d, must be in [1, %d]", n_plans, bsa::kMaxSchemes);
+  bsa::SchemeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  for (int c = 0; c < n_plans; ++c) {
+    bsa_status s = check_plan(plans[c]);
+    if (s != BSA_OK) return s;
+    const Geo& g = plans[c]->g;
+    const Geo& g0 = plans[0]->g;
+    if (g.B != g0.B || g.T != g0.T || g.H != g0.H || g.W != g0.W || g.Hd != g0.Hd ||
+        g.D != g0.D || g.n_text != g0.n_text || plans[c]->dtype != plans[0]->dtype)
+      return fail(BSA_ERR_INVALID_ARG,
+                  "candidate %d differs from candidate 0 in more than the block shape", c);
+    if (sics[c] == nullptr && g.nb > 0) return fail(BSA_ERR_INVALID_ARG, "SICS output %d is NULL", c);
+    a.g[c] = g;
+    a.sics[c] = sics[c];
+  }
+  if (x == nullptr) return fail(BSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(x)) return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  a.x = x;
+  a.as = as;
+  a.choice = choice;
+  a.n = n_plans;
+  const Geo& g0 = plans[0]->g;
+  if ((long long)g0.B * g0.Hd > 65535)
+    return fail(BSA_ERR_UNSUPPORTED, "batch * heads = %lld exceeds 65535", (long long)g0.B * g0.Hd);
+  if ((long long)g0.B * g0.Hd == 0) return BSA_OK;
+  cudaError_t e = bsa::launch_sics_schemes(a, plans[0]->dtype == BSA_BF16, (cudaStream_t)stream);
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "SICS kernel");
+}
+
 bsa_status bsa_check_status(bsa_plan_t p, void* stream) {
   bsa_status s = check_plan(p);
   if (s != BSA_OK) return s;

@@ -9,7 +9,21 @@ struct GatherArgs {
   const void* src[3];
   void* dst[3];      // unused in kPool
   float* cent[3];    // optional centroid outputs (kPermute, kPool)
+  float* sics[3];    // optional SICS outputs [B, Hd, nb] (kPermute, kPool, kPoolOrig)
   int ntensors;
+};
+
+// Aggregation evaluation of up to kMaxSchemes candidate blocking schemes of
+// one tensor in the original layout (every g[c] shares B, T, H, W, Hd, D,
+// n_text; only the block shape differs).
+constexpr int kMaxSchemes = 8;
+struct SchemeArgs {
+  Geo g[kMaxSchemes];
+  float* sics[kMaxSchemes];   // [B, Hd, nb_c] per candidate
+  const void* x;              // [B, Ntot, Hd, D]
+  double* as;                 // [n, B, Hd] or null
+  int32_t* choice;            // [B, Hd] or null
+  int n;
 };
 
 struct SelectArgs {
@@ -49,6 +63,7 @@ struct TileMaps {
 cudaError_t launch_permute(const Geo& g, bool is_bf16, const GatherArgs& a, cudaStream_t st);
 cudaError_t launch_unpermute(const Geo& g, bool is_bf16, const GatherArgs& a, cudaStream_t st);
 cudaError_t launch_pool(const Geo& g, bool is_bf16, const GatherArgs& a, cudaStream_t st);
+cudaError_t launch_sics_schemes(const SchemeArgs& a, bool is_bf16, cudaStream_t st);
 // select.cu
 size_t select_smem_bytes(int nb, int D);
 cudaError_t launch_select(const Geo& g, const SelectArgs& a, cudaStream_t st);

@@ -41,16 +41,42 @@ __device__ __forceinline__ void accumulate_vec(float* acc, const uint4& v) {
   }
 }
 
+template <typename T>
+__device__ __forceinline__ void to_float(const uint4& v, float* f) {
+  if constexpr (sizeof(T) == 2) {
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 t = __bfloat1622float2(p[i]);
+      f[2 * i] = t.x;
+      f[2 * i + 1] = t.y;
+    }
+  } else {
+    f[0] = __uint_as_float(v.x);
+    f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z);
+    f[3] = __uint_as_float(v.w);
+  }
+}
+
+// One CTA's work: tile (tensor, b, h, block j).  With a.sics[tensor] set it
+// also evaluates the intra-block estimator of SPADE §3.2, Eq. (4), the sum of
+// all pairwise cosine similarities of the block's valid rows, in the form
+// || sum_a q_a / |q_a| ||^2 (equal to Eq. (4) by expanding the square; a zero
+// row has no direction and contributes nothing).  The running sum of unit
+// rows is the r of the online form (Eq. (5)); squaring it once at the end
+// instead of accumulating the cross terms keeps every term of the fp32 sum
+// non-negative.
 template <typename T, int D, int MODE>
-__global__ void __launch_bounds__(kGatherThreads) gather_kernel(Geo g, GatherArgs a) {
+__device__ __forceinline__ void gather_block(const Geo& g, const void* src_ptr, void* dst_ptr,
+                                             float* cent_ptr, float* sics_ptr, int j, int h, int b) {
   constexpr int E = 16 / (int)sizeof(T);  // elements per 16-byte vector
   constexpr int V = D / E;                // vectors per row
   constexpr int R = kGatherThreads / V;   // rows per pass
   __shared__ int s_tok[256];
   __shared__ float s_red[R * D];
+  __shared__ float s_warp[kGatherThreads / 32];
 
-  const int j = blockIdx.x, h = blockIdx.y;
-  const int tensor = blockIdx.z % a.ntensors, b = blockIdx.z / a.ntensors;
   const int tid = threadIdx.x, row0 = tid / V, vec = tid % V;
 
   for (int s = tid; s < g.bs; s += kGatherThreads) s_tok[s] = (int)slot_token(g, j, s);
@@ -58,13 +84,14 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(Geo g, GatherArg
 
   const long long blk_row0 = (long long)(b * g.Hd + h) * g.npad_tot + (long long)j * g.bs;
   const long long tok_base = (long long)b * g.n_tot;
-  float* cent = (MODE != kUnpermute && j < g.nb) ? a.cent[tensor] : nullptr;
-  float acc[E];
+  float* cent = (MODE != kUnpermute && j < g.nb) ? cent_ptr : nullptr;
+  float* sics = (MODE != kUnpermute && j < g.nb) ? sics_ptr : nullptr;
+  float acc[E], racc[E];
 #pragma unroll
-  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  for (int e = 0; e < E; ++e) acc[e] = racc[e] = 0.f;
 
-  const uint4* src = reinterpret_cast<const uint4*>(a.src[tensor]);
-  uint4* dst = reinterpret_cast<uint4*>(a.dst[tensor]);
+  const uint4* src = reinterpret_cast<const uint4*>(src_ptr);
+  uint4* dst = reinterpret_cast<uint4*>(dst_ptr);
   for (int s0 = 0; s0 < g.bs; s0 += R * kUnroll) {
     uint4 buf[kUnroll];
     int tok[kUnroll];
@@ -86,6 +113,19 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(Geo g, GatherArg
       if (MODE == kPermute && tok[u] >= -1) dst[(blk_row0 + s) * V + vec] = buf[u];
       if (MODE == kUnpermute && tok[u] >= 0) dst[((tok_base + tok[u]) * g.Hd + h) * V + vec] = buf[u];
       if (MODE != kUnpermute && cent != nullptr && tok[u] >= 0) accumulate_vec<T>(acc, buf[u]);
+      if (MODE != kUnpermute && sics != nullptr) {
+        // Every lane takes part (pad and out-of-range rows hold zeros): the V
+        // lanes of one row are an aligned group of the warp.
+        float f[E], ss = 0.f;
+        to_float<T>(buf[u], f);
+#pragma unroll
+        for (int e = 0; e < E; ++e) ss = fmaf(f[e], f[e], ss);
+#pragma unroll
+        for (int o = V / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) racc[e] = fmaf(f[e], inv, racc[e]);
+      }
     }
   }
 
@@ -100,6 +140,196 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(Geo g, GatherArg
       cent[((long long)(b * g.Hd + h) * g.nb + j) * D + tid] = sum / n;
     }
   }
+
+  if (MODE != kUnpermute && sics != nullptr) {
+    __syncthreads();  // s_red is reused after the centroid reduction
+#pragma unroll
+    for (int e = 0; e < E; ++e) s_red[row0 * D + vec * E + e] = racc[e];
+    __syncthreads();
+    float r2 = 0.f;
+    if (tid < D) {
+      float r = 0.f;
+      for (int rr = 0; rr < R; ++rr) r += s_red[rr * D + tid];
+      r2 = r * r;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) r2 += __shfl_xor_sync(0xffffffffu, r2, o);
+    if ((tid & 31) == 0) s_warp[tid >> 5] = r2;
+    __syncthreads();
+    if (tid == 0) {
+      float t = 0.f;
+      for (int w = 0; w < D / 32; ++w) t += s_warp[w];
+      sics[(long long)(b * g.Hd + h) * g.nb + j] = t;
+    }
+  }
+}
+
+template <typename T, int D, int MODE>
+__global__ void __launch_bounds__(kGatherThreads) gather_kernel(Geo g, GatherArgs a) {
+  // Constant-index reads of the pointer arrays (a dynamic index would copy
+  // the argument block to local memory).
+  const int t = blockIdx.z % a.ntensors;
+  const void* src = t == 0 ? a.src[0] : t == 1 ? a.src[1] : a.src[2];
+  void* dst = t == 0 ? a.dst[0] : t == 1 ? a.dst[1] : a.dst[2];
+  float* cent = t == 0 ? a.cent[0] : t == 1 ? a.cent[1] : a.cent[2];
+  float* sics = t == 0 ? a.sics[0] : t == 1 ? a.sics[1] : a.sics[2];
+  gather_block<T, D, MODE>(g, src, dst, cent, sics, blockIdx.x, blockIdx.y, blockIdx.z / a.ntensors);
+}
+
+// Aggregation evaluation (SPADE §3.2): SICS of every block of every candidate
+// blocking scheme, read from the original layout.  One warp per (b, h,
+// candidate, block): the online form of Eq. (5), a running sum of unit rows
+// per lane, with no block barrier.  A lane holds kSicsChunks 16-byte pieces of
+// a row, so L lanes share one row of D elements and one warp step covers
+// RPI = 32 / L rows; piece k of lane v is row bytes [(k L + v) 16, +16), so
+// every copy instruction reads whole 128-byte segments.  Each warp streams its
+// rows through a private kSicsStages-deep shared-memory ring with 16-byte
+// cp.async copies (rows past the block's end are zero-filled, not read), so
+// that kSicsStages steps per warp are in flight without holding registers.
+// Warps are numbered head-major, then candidate, then block: the candidates
+// of one head run back to back and re-read its rows from L2 (HBM traffic is
+// one read of x whatever the number of candidates).
+constexpr int kSicsWarps = 4;
+constexpr int kSicsStages = 4;
+constexpr int kSicsChunks = 4;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kSicsWarps * 32, 4) sics_schemes_kernel(SchemeArgs s, int per_bh,
+                                                                        long long n_tasks) {
+  constexpr int E = 16 / (int)sizeof(T);          // elements per 16-byte piece
+  constexpr int C = kSicsChunks;
+  constexpr int L = D / (E * C);                  // lanes per row
+  constexpr int RPI = 32 / L;                     // rows per warp step
+  static_assert(L >= 1 && L <= 32 && 32 % L == 0, "row split");
+  __shared__ __align__(16) uint4 s_ring[kSicsWarps][kSicsStages][C][32];
+  const int warp = threadIdx.x >> 5;
+  const long long task = (long long)blockIdx.x * kSicsWarps + warp;
+  if (task >= n_tasks) return;
+  const int lane = threadIdx.x & 31, sub = lane / L, vec = lane % L;
+  const int bh = (int)(task / per_bh);
+  int j = (int)(task % per_bh), c = 0;
+  while (j >= s.g[c].nb) j -= s.g[c++].nb;
+  const Geo& g = s.g[c];
+  const int b = bh / g.Hd, h = bh % g.Hd;
+  const int xb = j % g.nbx, yb = (j / g.nbx) % g.nby, tb = j / (g.nbx * g.nby);
+  const int t0 = tb * g.bf, y0 = yb * g.br, x0 = xb * g.bc;
+  const int vt = min(g.bf, g.T - t0), vy = min(g.br, g.H - y0), vx = min(g.bc, g.W - x0);
+  const int n = vt * vy * vx;
+  const int n_steps = (n + RPI - 1) / RPI;
+  // (dt, dy, dx) of this lane's next row (row `sub`, then +RPI per step) and
+  // the row's address, advanced with carries instead of divisions.
+  const long long sx = (long long)g.Hd * L * C;          // 16-byte pieces per token
+  const long long sy = sx * g.W, st = sy * g.H;
+  const uint4* first = reinterpret_cast<const uint4*>(s.x) +
+                       ((long long)b * g.n_tot * g.Hd + h) * (L * C) + vec +
+                       ((long long)t0 * g.H + y0) * sy + (long long)x0 * sx;
+  const uint4* ptr = first;
+  int dx = 0, dy = 0, dt = 0;
+  auto advance = [&](int k) {
+    dx += k;
+    ptr += k * sx;
+    while (dx >= vx && dt < vt) {
+      dx -= vx;
+      ptr += sy - vx * sx;
+      if (++dy >= vy) {
+        dy = 0;
+        ++dt;
+        ptr += st - vy * sy;
+      }
+    }
+  };
+  advance(sub);
+  const uint32_t ring = smem_addr(&s_ring[warp][0][0][lane]);
+  auto issue = [&](int step) {   // steps are issued in order 0, 1, 2, ...
+    const bool ok = step * RPI + sub < n;
+    const uint32_t dst = ring + (uint32_t)((step % kSicsStages) * C * 32 * 16);
+#pragma unroll
+    for (int k = 0; k < C; ++k)
+      cp_async16(dst + k * 32 * 16, ok ? ptr + k * L : first, ok ? 16u : 0u);
+    advance(RPI);
+  };
+#pragma unroll
+  for (int k = 0; k < kSicsStages - 1; ++k) {
+    if (k < n_steps) issue(k);
+    cp_async_commit();
+  }
+  float2 racc[C * E / 2];
+#pragma unroll
+  for (int e = 0; e < C * E / 2; ++e) racc[e] = make_float2(0.f, 0.f);
+  for (int i = 0; i < n_steps; ++i) {
+    if (i + kSicsStages - 1 < n_steps) issue(i + kSicsStages - 1);
+    cp_async_commit();
+    cp_async_wait<kSicsStages - 1>();   // this lane's copies of step i have landed
+    float2 f[C * E / 2];
+#pragma unroll
+    for (int k = 0; k < C; ++k) to_float<T>(s_ring[warp][i % kSicsStages][k][lane],
+                                            reinterpret_cast<float*>(f + k * E / 2));
+    float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int e = 0; e < C * E / 2; ++e) ss2 = fma2(f[e], f[e], ss2);
+    float ss = ss2.x + ss2.y;
+#pragma unroll
+    for (int o = L / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
+    const float2 inv2 = make_float2(inv, inv);
+#pragma unroll
+    for (int e = 0; e < C * E / 2; ++e) racc[e] = fma2(f[e], inv2, racc[e]);
+  }
+  cp_async_wait<0>();
+  // r = sum over the RPI row groups; |r|^2 = sum over the L lanes of one group
+  float r2 = 0.f;
+#pragma unroll
+  for (int e = 0; e < C * E / 2; ++e) {
+    float rx = racc[e].x, ry = racc[e].y;
+#pragma unroll
+    for (int o = L; o < 32; o <<= 1) {
+      rx += __shfl_xor_sync(0xffffffffu, rx, o);
+      ry += __shfl_xor_sync(0xffffffffu, ry, o);
+    }
+    r2 = fmaf(rx, rx, r2);
+    r2 = fmaf(ry, ry, r2);
+  }
+#pragma unroll
+  for (int o = L / 2; o >= 1; o >>= 1) r2 += __shfl_xor_sync(0xffffffffu, r2, o);
+  if (lane == 0) s.sics[c][(long long)bh * g.nb + j] = r2;
+}
+
+// Aggregation score AS(x | scheme c) = sum over the video blocks of SICS
+// (SPADE §3.2, Eq. (3)), summed in double in a fixed order, and the
+// per-(b, h) choice of the scheme with the largest AS (lowest candidate
+// index among equal scores).  One warp per (b, h).
+__global__ void __launch_bounds__(128) aggregate_kernel(SchemeArgs s, int BH) {
+  const int bh = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (bh >= BH) return;
+  double best = 0.0;
+  int arg = 0;
+  for (int c = 0; c < s.n; ++c) {
+    const int nb = s.g[c].nb;
+    const float* src = s.sics[c] + (long long)bh * nb;
+    double t = 0.0;
+    for (int jj = lane; jj < nb; jj += 32) t += (double)src[jj];
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (s.as != nullptr && lane == 0) s.as[(long long)c * BH + bh] = t;
+    if (c == 0 || t > best) {
+      best = t;
+      arg = c;
+    }
+  }
+  if (s.choice != nullptr && lane == 0) s.choice[bh] = arg;
 }
 
 template <typename T, int MODE>
@@ -138,6 +368,31 @@ cudaError_t launch_pool_orig(const Geo& g, bool is_bf16, const GatherArgs& a, cu
 cudaError_t launch_pool(const Geo& g, bool is_bf16, const GatherArgs& a, cudaStream_t st) {
   return is_bf16 ? launch_gather_t<__nv_bfloat16, kPool>(g, a, g.nb, st)
                  : launch_gather_t<float, kPool>(g, a, g.nb, st);
+}
+
+cudaError_t launch_sics_schemes(const SchemeArgs& a, bool is_bf16, cudaStream_t st) {
+  const Geo& g0 = a.g[0];
+  int per_bh = 0;
+  for (int c = 0; c < a.n; ++c) per_bh += a.g[c].nb;
+  const int BH = g0.B * g0.Hd;
+  const long long n_tasks = (long long)per_bh * BH;
+  if (n_tasks > 0) {
+    const long long grid = (n_tasks + kSicsWarps - 1) / kSicsWarps;
+    if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const dim3 gd((unsigned)grid), bd(kSicsWarps * 32);
+    if (is_bf16) {
+      if (g0.D == 128) sics_schemes_kernel<__nv_bfloat16, 128><<<gd, bd, 0, st>>>(a, per_bh, n_tasks);
+      else sics_schemes_kernel<__nv_bfloat16, 64><<<gd, bd, 0, st>>>(a, per_bh, n_tasks);
+    } else {
+      if (g0.D == 128) sics_schemes_kernel<float, 128><<<gd, bd, 0, st>>>(a, per_bh, n_tasks);
+      else sics_schemes_kernel<float, 64><<<gd, bd, 0, st>>>(a, per_bh, n_tasks);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (a.as != nullptr || a.choice != nullptr)
+    aggregate_kernel<<<(BH + 3) / 4, 128, 0, st>>>(a, BH);
+  return cudaGetLastError();
 }
 
 }  // namespace bsa

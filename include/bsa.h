@@ -146,6 +146,36 @@ bsa_status bsa_permute_qkv(bsa_plan_t plan, const void* q, const void* k,
 bsa_status bsa_centroids(bsa_plan_t plan, const void* q, const void* k,
                          float* q_cent, float* k_cent, void* stream);
 
+/* bsa_sics — the intra-block estimator of SPADE §3.2, Eq. (4): for every
+ * video block of the plan's blocking scheme, the sum over all ordered pairs
+ * (a, b) of the block's valid rows (diagonal included) of the cosine
+ * similarity x_a . x_b / (|x_a| |x_b|).  It equals |sum_a x_a/|x_a| |^2 and
+ * lies in [0, n^2] for a block of n valid rows; a zero row has no direction
+ * and contributes nothing.  Computed in fp32 (rows widened exactly from the
+ * plan dtype).  Text tokens belong to no 3D block and take no part.
+ *   x     [B, Ntot, Hd, D] original order (read only)
+ *   sics  [B, Hd, nb] float out */
+bsa_status bsa_sics(bsa_plan_t plan, const void* x, float* sics, void* stream);
+
+/* bsa_aggregation_scores — aggregation evaluation and blocking-scheme choice
+ * (SPADE §3.2): for each candidate plan c (a blocking scheme), the SICS of
+ * every video block, the Aggregation Score AS(x | c) = sum of SICS over the
+ * video blocks (Eq. (3)), and per (b, h) the candidate with the largest AS
+ * (the Selected Blocking Scheme; the lowest c among equal scores).
+ *   plans   host array of n_plans (1..8) plans on the current device that
+ *           agree in batch, T, H, W, heads, head_dim, n_text and dtype
+ *   x       [B, Ntot, Hd, D] original order (read only)
+ *   sics    host array of n_plans device pointers, sics[c] = [B, Hd, nb_c]
+ *           float out (required: it also carries AS's terms)
+ *   as      [n_plans, B, Hd] double out, optional (NULL = skip); the fp32
+ *           SICS values summed in double in a fixed order
+ *   choice  [B, Hd] int32 out, optional (NULL = skip)
+ * One launch evaluates all candidates, with the candidates of a head
+ * scheduled together so that the head's rows are read from HBM once. */
+bsa_status bsa_aggregation_scores(const bsa_plan_t* plans, int n_plans,
+                                  const void* x, float* const* sics,
+                                  double* as, int32_t* choice, void* stream);
+
 /* bsa_unpermute — restore blocked output to the original token order (SPADE
  * §3.3, "output blocks are restored to the original layout"); pad slots are
  * dropped.   o_blk [B, Hd, Npad_tot, D] -> o [B, Ntot, Hd, D]. */

@@ -101,3 +101,45 @@ def custom_workload(name, B, T, H, W, bf, br, bc, Hd, D, n_text, dtype, mode, pa
     w = synthetic.Workload(name, B, T, H, W, bf, br, bc, Hd, D, dtype, mode, [param] * Hd,
                            n_text=n_text, qk_std=3.0 if dtype == "bf16" else None)
     return w
+
+
+# ------------------------------------------------------------------ SICS --
+U32 = 2.0 ** -24   # unit roundoff of fp32
+
+
+def valid_counts(g) -> np.ndarray:
+    """[nb] number of valid tokens of every video block."""
+    j = np.arange(g.nb)
+    tb, yb, xb = j // (g.nby * g.nbx), (j // g.nbx) % g.nby, j % g.nbx
+    vt = np.minimum(g.bf, g.T - tb * g.bf)
+    vy = np.minimum(g.br, g.H - yb * g.br)
+    vx = np.minimum(g.bc, g.W - xb * g.bc)
+    return (vt * vy * vx).astype(np.float64)
+
+
+def sics_tol(g, ref) -> np.ndarray:
+    """Forward error bound of the fp32 SICS kernel, per block ([..., nb]).
+
+    The kernel forms r = sum_a x_a * rsqrt(|x_a|^2) and returns |r|^2, all in
+    fp32, for n <= bs valid rows of D elements.  Each unit row carries a
+    relative error of at most (D/2 + 3) u (the D-term sum of squares, rsqrtf's
+    2 ulp, the product); the n-term sums of r add n u times sum_a |xhat_a|,
+    whose norm is at most n.  So |delta r| <= n (n + D/2 + 3) u =: e and
+    |delta |r|^2| <= 2 |r| e + e^2 + (D + 1) u |r|^2, with |r| = sqrt(SICS).
+    """
+    n = valid_counts(g)
+    e = n * (n + g.D / 2 + 3) * U32
+    r = np.sqrt(np.maximum(ref, 0.0))
+    return 2 * r * e + e * e + (g.D + 1) * U32 * ref + 1e-6
+
+
+def check_sics(g, gpu, ref, what=""):
+    """SICS within the derived bound; returns (max_abs_err, max err/bound)."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    assert np.all(np.isfinite(gpu)), f"{what}: non-finite SICS"
+    tol = sics_tol(g, ref)
+    err = np.abs(gpu - ref)
+    worst = float((err / tol).max()) if err.size else 0.0
+    assert worst <= 1.0, f"{what}: SICS error {float(err.max()):.3e} above its bound (x{worst:.2f})"
+    return (float(err.max()) if err.size else 0.0), worst

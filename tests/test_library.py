@@ -74,6 +74,19 @@ def test_null_arguments_are_rejected(lib):
     assert lib.bsa_plan_destroy(None) == 0
 
 
+def test_aggregation_scores_rejects_bad_candidate_lists(lib):
+    P = ctypes.c_void_p
+    lib.bsa_aggregation_scores.argtypes = [P, ctypes.c_int, P, P, P, P, P]
+    lib.bsa_aggregation_scores.restype = ctypes.c_int
+    plans = (P * 9)()
+    outs = (P * 9)()
+    assert lib.bsa_aggregation_scores(None, 1, None, outs, None, None, None) == 1
+    assert lib.bsa_aggregation_scores(plans, 1, None, None, None, None, None) == 1
+    for n in (0, 9, -1):
+        assert lib.bsa_aggregation_scores(plans, n, None, outs, None, None, None) == 1
+        assert "n_plans" in lib.bsa_last_error_string().decode()
+
+
 def test_plan_create_without_device_reports_cuda_error(lib):
     import torch
     if torch.cuda.is_available():
