@@ -53,6 +53,8 @@ def _load():
         lib.orc_k_for_density.restype = ctypes.c_int
         lib.orc_select.argtypes = [P, P, ctypes.c_int, P, ctypes.c_int, P, P, P]
         lib.orc_attention.argtypes = [P, P, P, P, P, P, ctypes.c_int, P, ctypes.c_longlong, P]
+        lib.orc_select_union.argtypes = [P, P, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int, P,
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_longlong, P, P, P]
         lib.orc_sics.argtypes = [P, P, P]
         lib.orc_sics_online.argtypes = [P, P, P]
         lib.orc_aggregation_score.argtypes = [P, P, P]
@@ -150,6 +152,32 @@ def select(g: Geometry, p, mode: int, params, kmax: int | None = None):
     tie = np.zeros((g.B, g.Hd, g.nb), dtype=np.int32)
     _load().orc_select(_ptr(g.arr), _ptr(p), int(mode), _ptr(params), int(kmax),
                        _ptr(idx), _ptr(cnt), _ptr(tie))
+    return idx, cnt, tie
+
+
+def select_union(g: Geometry, p, mode: int, params, window=(-1, -1), sink_tokens=0,
+                 intra=None, intra_mode: int = 0, intra_params=None, kmax: int | None = None):
+    """Lists of the mask union (SPADE §3.3): inter Top-K/Top-P of p, united with a
+    sliding window over the block sequence, the attention-sink blocks and the
+    intra-score selection broadcast over query blocks.  Returns (idx, cnt, tie)."""
+    params = np.ascontiguousarray(params, dtype=np.float64)
+    assert params.shape == (g.Hd,)
+    if kmax is None:
+        kmax = g.nb + g.nb_text
+    p = np.ascontiguousarray(p, dtype=np.float64)
+    ip = None
+    if intra is not None:
+        intra = np.ascontiguousarray(intra, dtype=np.float64)
+        assert intra.shape == (g.B, g.Hd, g.nb)
+        ip = np.ascontiguousarray(intra_params, dtype=np.float64)
+        assert ip.shape == (g.Hd,)
+    idx = np.full((g.B, g.Hd, g.nb, kmax), -1, dtype=np.int32)
+    cnt = np.zeros((g.B, g.Hd, g.nb), dtype=np.int32)
+    tie = np.zeros((g.B, g.Hd, g.nb), dtype=np.int32)
+    _load().orc_select_union(_ptr(g.arr), _ptr(p), int(mode), _ptr(params), int(kmax),
+                             None if intra is None else _ptr(intra), int(intra_mode),
+                             None if ip is None else _ptr(ip), int(window[0]), int(window[1]),
+                             int(sink_tokens), _ptr(idx), _ptr(cnt), _ptr(tie))
     return idx, cnt, tie
 
 

@@ -37,6 +37,12 @@
 //      text key blocks; text query tokens attend every token.
 //   R9 lists are stored in ascending block id, text blocks last.
 //   R15 SICS: a zero vector has no direction and contributes nothing.
+//   R18 local window: key blocks j with i - left <= j <= i + right over the
+//       block sequence; a negative side is unbounded; (-1, -1) = no window.
+//   R19 attention sink: the key blocks holding any of the first S tokens of
+//       the original sequence.
+//   R20 intra scores: one per key block, broadcast to every query block of
+//       the head; selected by the Top-K / Top-P rule on the scores.
 //
 // Geometry array g[10] = {B, T, H, W, bf, br, bc, Hd, D, n_text}.
 
@@ -122,6 +128,53 @@ std::vector<long long> block_tokens(const Geom& G, long long j) {
       out.push_back(G.n_video + u);
   }
   return out;
+}
+
+// Top-K / Top-P rule over one row of nonnegative weights v[0..nb) (R5-R7,
+// R12): order by v descending, then index ascending; Top-K keeps
+// k_for_density(param) entries, Top-P the smallest m >= 1 whose prefix sum
+// reaches param * total.  `chosen` gets the kept indices; `tie` is set when
+// the cut sits on a near-tie (1e-5 relative).
+int k_for_density_(double rho, long long nb) {
+  long long k = (long long)std::ceil(rho * (double)nb - 1e-9);
+  if (k < 1) k = 1;
+  if (k > nb) k = nb;
+  return (int)k;
+}
+
+void select_rule(const double* v, long long nb, int mode, double param, double total,
+                 std::vector<long long>& chosen, int& tie) {
+  std::vector<long long> order(nb);
+  for (long long j = 0; j < nb; ++j) order[j] = j;
+  std::sort(order.begin(), order.end(), [&](long long a, long long b) {
+    if (v[a] != v[b]) return v[a] > v[b];
+    return a < b;
+  });
+  long long m;
+  if (mode == 0) {
+    m = k_for_density_(param, nb);
+    if (m < nb) {
+      double a = v[order[m - 1]], b = v[order[m]];
+      if (std::fabs(a - b) <= 1e-5 * std::fabs(a)) tie = 1;
+    }
+  } else {
+    const double target = param * total;
+    double cum = 0.0, before = 0.0;
+    m = 0;
+    while (m < nb) {
+      before = cum;
+      cum += v[order[m]];
+      ++m;
+      if (cum >= target) break;
+    }
+    if (std::fabs(before - target) <= 1e-5 * target) tie = 1;
+    if (std::fabs(cum - target) <= 1e-5 * target) tie = 1;
+    if (m < nb) {
+      double a = v[order[m - 1]], b = v[order[m]];
+      if (std::fabs(a - b) <= 1e-5 * std::fabs(a)) tie = 1;
+    }
+  }
+  chosen.assign(order.begin(), order.begin() + m);
 }
 
 }  // namespace
@@ -226,12 +279,7 @@ void orc_scores(const int* g, const double* qc, const double* kc, double* p) {
 
 // Number of key blocks a density keeps (R5; the blog's "fraction of key
 // blocks each query block keeps").
-int orc_k_for_density(double rho, int nb) {
-  long long k = (long long)std::ceil(rho * (double)nb - 1e-9);
-  if (k < 1) k = 1;
-  if (k > nb) k = nb;
-  return (int)k;
-}
+int orc_k_for_density(double rho, int nb) { return k_for_density_(rho, nb); }
 
 // Top-K / Top-P selection (SPADE §3.1 "Top-K/Top-P mode"; §3.3 "Scores are
 // filtered by Top-K or Top-P"; inter-top value = "Top-P cumulative threshold
@@ -244,38 +292,9 @@ void orc_select(const int* g, const double* p, int mode, const double* params,
   Geom G = make_geom(g);
   parallel_for(G.B * G.Hd * G.nb, [&](long long row) {
     long long h = (row / G.nb) % G.Hd;
-    const double* pr = p + row * G.nb;
-    std::vector<long long> order(G.nb);
-    for (long long j = 0; j < G.nb; ++j) order[j] = j;
-    std::sort(order.begin(), order.end(), [&](long long a, long long b) {
-      if (pr[a] != pr[b]) return pr[a] > pr[b];
-      return a < b;
-    });
-    long long m;
+    std::vector<long long> chosen;
     int is_tie = 0;
-    if (mode == 0) {
-      m = orc_k_for_density(params[h], (int)G.nb);
-      if (m < G.nb) {
-        double a = pr[order[m - 1]], b = pr[order[m]];
-        if (std::fabs(a - b) <= 1e-5 * std::fabs(a)) is_tie = 1;
-      }
-    } else {
-      double tau = params[h], cum = 0.0, before = 0.0;
-      m = 0;
-      while (m < G.nb) {
-        before = cum;
-        cum += pr[order[m]];
-        ++m;
-        if (cum >= tau) break;
-      }
-      if (std::fabs(before - tau) <= 1e-5 * tau) is_tie = 1;
-      if (std::fabs(cum - tau) <= 1e-5 * tau) is_tie = 1;
-      if (m < G.nb) {
-        double a = pr[order[m - 1]], b = pr[order[m]];
-        if (std::fabs(a - b) <= 1e-5 * std::fabs(a)) is_tie = 1;
-      }
-    }
-    std::vector<long long> chosen(order.begin(), order.begin() + m);
+    select_rule(p + row * G.nb, G.nb, mode, params[h], 1.0, chosen, is_tie);
     std::sort(chosen.begin(), chosen.end());
     int* out = idx + row * kmax;
     long long c = 0;
@@ -283,6 +302,73 @@ void orc_select(const int* g, const double* p, int mode, const double* params,
     for (long long t = 0; t < G.nb_text; ++t) out[c++] = (int)(G.nb + t);
     cnt[row] = (int)c;
     tie[row] = is_tie;
+  });
+}
+
+// Block lists of the mask union (SPADE §3.3: "intra scores are broadcast and
+// OR-combined with inter scores.  The result is united with local-window and
+// attention-sink masks"; §3.2 policy: local-window length, intra-top value,
+// inter-top value; §3.1 attention-sink length).  Per video query block i of
+// head h the list holds, in ascending id, the union of
+//   inter:  the Top-K / Top-P selection of p[b,h,i,:] (as orc_select);
+//   window: key blocks j with i - win_left <= j <= i + win_right (R18: a
+//           sliding window over the block sequence, (left, right) as in
+//           LongLive's window_size; a negative side is unbounded, and
+//           (-1, -1) turns the window off);
+//   sink:   key blocks holding any of the first sink_tokens tokens of the
+//           original sequence (R19);
+//   intra:  when intra != NULL and intra_params[h] > 0, the key blocks that
+//           the same rule selects from the intra scores intra[b,h,:] (R20:
+//           one score per key block, broadcast to every query block); Top-P
+//           takes the shortest descending prefix whose sum reaches
+//           tau * (sum of all scores);
+// then the text key blocks.  tie[] flags rows whose inter selection, or
+// whose head's intra selection, sits on a tie (R12).
+void orc_select_union(const int* g, const double* p, int mode, const double* params, int kmax,
+                      const double* intra, int intra_mode, const double* intra_params,
+                      int win_left, int win_right, long long sink_tokens,
+                      int* idx, int* cnt, int* tie) {
+  Geom G = make_geom(g);
+  std::vector<char> sink(G.nb, 0);
+  for (long long j = 0; j < G.nb; ++j) {
+    std::vector<long long> toks = block_tokens(G, j);
+    for (long long t : toks)
+      if (t < sink_tokens) sink[j] = 1;
+  }
+  std::vector<std::vector<char>> intra_set(G.B * G.Hd, std::vector<char>(G.nb, 0));
+  std::vector<int> intra_tie(G.B * G.Hd, 0);
+  if (intra != nullptr && intra_params != nullptr) {
+    for (long long bh = 0; bh < G.B * G.Hd; ++bh) {
+      const double prm = intra_params[bh % G.Hd];
+      if (!(prm > 0.0)) continue;
+      const double* v = intra + bh * G.nb;
+      double total = 0.0;
+      for (long long j = 0; j < G.nb; ++j) total += v[j];
+      std::vector<long long> chosen;
+      select_rule(v, G.nb, intra_mode, prm, total, chosen, intra_tie[bh]);
+      for (long long j : chosen) intra_set[bh][j] = 1;
+    }
+  }
+  const bool window = !(win_left < 0 && win_right < 0);
+  parallel_for(G.B * G.Hd * G.nb, [&](long long row) {
+    long long bh = row / G.nb, h = bh % G.Hd, i = row % G.nb;
+    std::vector<long long> chosen;
+    int is_tie = 0;
+    select_rule(p + row * G.nb, G.nb, mode, params[h], 1.0, chosen, is_tie);
+    std::vector<char> take(G.nb, 0);
+    for (long long j : chosen) take[j] = 1;
+    for (long long j = 0; j < G.nb; ++j) {
+      if (window && (win_left < 0 || j >= i - win_left) && (win_right < 0 || j <= i + win_right))
+        take[j] = 1;
+      if (sink[j] || intra_set[bh][j]) take[j] = 1;
+    }
+    int* out = idx + row * kmax;
+    long long c = 0;
+    for (long long j = 0; j < G.nb; ++j)
+      if (take[j]) out[c++] = (int)j;
+    for (long long t = 0; t < G.nb_text; ++t) out[c++] = (int)(G.nb + t);
+    cnt[row] = (int)c;
+    tie[row] = is_tie | intra_tie[bh];
   });
 }
 

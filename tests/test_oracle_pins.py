@@ -334,3 +334,107 @@ def test_aggregation_score_and_scheme_choice():
     for gi, g in enumerate(geoms):
         np.testing.assert_allclose(scores[gi], orc.sics(g, x).sum(-1), rtol=1e-13)
     assert np.all(scores[choice[0], 0, np.arange(3)] >= scores.max(0)[0] - 1e-12)
+
+
+# ------------------------------------------------ mask-union pins (SPADE §3.3)
+def _inter_sets(g, p, mode, params):
+    idx, cnt, _ = orc.select(g, p, mode, params)
+    return {(b, h, i): set(int(j) for j in idx[b, h, i, :cnt[b, h, i] - g.nb_text])
+            for b in range(g.B) for h in range(g.Hd) for i in range(g.nb)}
+
+
+def _max_mass_prefix(v, tau_total):
+    """Smallest m whose best m-subset reaches tau_total, by exhaustive search;
+    returns that subset (the m largest, ties to the lower index)."""
+    nb = len(v)
+    for m in range(1, nb + 1):
+        best = max(itertools.combinations(range(nb), m), key=lambda c: (sum(v[j] for j in c),
+                                                                        [-j for j in c]))
+        if sum(v[j] for j in best) >= tau_total:
+            return set(best)
+    return set(range(nb))
+
+
+def test_union_window_predicate():
+    g = orc.Geometry(**RAGGED)
+    p = _rand_p(g, 20)
+    inter = _inter_sets(g, p, 0, [0.25, 0.25])
+    for window in [(0, 0), (1, 2), (2, -1), (-1, 1), (-1, -1), (100, 100)]:
+        idx, cnt, _ = orc.select_union(g, p, 0, [0.25, 0.25], window=window)
+        for (b, h, i), s in inter.items():
+            lo = -10**9 if window[0] < 0 else i - window[0]
+            hi = 10**9 if window[1] < 0 else i + window[1]
+            win = set() if window == (-1, -1) else {j for j in range(g.nb) if lo <= j <= hi}
+            expect = sorted(s | win) + list(range(g.nb, g.nb + g.nb_text))
+            assert list(idx[b, h, i, :cnt[b, h, i]]) == expect, (window, b, h, i)
+
+
+def test_union_sink_blocks_hold_the_first_tokens():
+    g = orc.Geometry(**RAGGED)
+    p = _rand_p(g, 21)
+    inter = _inter_sets(g, p, 0, [0.25, 0.25])
+    tab = token_table(g)[:g.nb]
+    for sink in [0, 1, g.W, g.W + 1, g.H * g.W, g.n_video, g.n_tot]:
+        blocks = {j for j in range(g.nb) if np.any((tab[j] >= 0) & (tab[j] < sink))}
+        idx, cnt, _ = orc.select_union(g, p, 0, [0.25, 0.25], sink_tokens=sink)
+        for (b, h, i), s in inter.items():
+            assert list(idx[b, h, i, :cnt[b, h, i] - g.nb_text]) == sorted(s | blocks), sink
+    assert {j for j in range(g.nb) if np.any((tab[j] >= 0) & (tab[j] < 1))} == {0}
+
+
+@pytest.mark.parametrize("intra_mode,iparams", [(0, [0.25, 0.5]), (1, [0.3, 0.7]), (0, [1.0, 0.0])])
+def test_union_intra_selection_broadcast(intra_mode, iparams):
+    g = orc.Geometry(**RAGGED)                       # nb = 8
+    p = _rand_p(g, 22)
+    inter = _inter_sets(g, p, 1, [0.5, 0.8])
+    v = np.random.default_rng(23).random((g.B, g.Hd, g.nb)) * 50.0
+    idx, cnt, tie = orc.select_union(g, p, 1, [0.5, 0.8], intra=v, intra_mode=intra_mode,
+                                     intra_params=iparams)
+    for b in range(g.B):
+        for h in range(g.Hd):
+            row = v[b, h]
+            if iparams[h] <= 0:
+                isel = set()
+            elif intra_mode == 0:
+                k = orc.k_for_density(iparams[h], g.nb)
+                isel = set(sorted(range(g.nb), key=lambda j: (-row[j], j))[:k])
+            else:
+                isel = _max_mass_prefix(row, iparams[h] * row.sum())
+            for i in range(g.nb):
+                got = list(idx[b, h, i, :cnt[b, h, i] - g.nb_text])
+                assert got == sorted(inter[(b, h, i)] | isel), (b, h, i)
+
+
+def test_union_of_everything_and_dense_cases():
+    g = orc.Geometry(**dict(RAGGED, B=1))
+    p = _rand_p(g, 24)
+    v = np.random.default_rng(25).random((g.B, g.Hd, g.nb))
+    full = list(range(g.nb + g.nb_text))
+    # any single source at full strength gives dense rows
+    for kw in [dict(window=(-1, 10**6)), dict(window=(10**6, -1)), dict(sink_tokens=g.n_video),
+               dict(intra=v, intra_mode=0, intra_params=[1.0, 1.0]),
+               dict(intra=v, intra_mode=1, intra_params=[1.0, 1.0])]:
+        idx, cnt, _ = orc.select_union(g, p, 0, [0.125, 0.125], **kw)
+        assert np.all(cnt == g.nb + g.nb_text)
+        assert list(idx[0, 1, 3, :cnt[0, 1, 3]]) == full
+    # the union is the OR of the separately computed unions
+    parts = [orc.select_union(g, p, 0, [0.125, 0.25], window=(1, 0)),
+             orc.select_union(g, p, 0, [0.125, 0.25], sink_tokens=9),
+             orc.select_union(g, p, 0, [0.125, 0.25], intra=v, intra_params=[0.25, 0.25])]
+    idx, cnt, _ = orc.select_union(g, p, 0, [0.125, 0.25], window=(1, 0), sink_tokens=9, intra=v,
+                                   intra_params=[0.25, 0.25])
+    for h in range(g.Hd):
+        for i in range(g.nb):
+            u = set()
+            for pi, pc, _ in parts:
+                u |= set(pi[0, h, i, :pc[0, h, i]].tolist())
+            assert list(idx[0, h, i, :cnt[0, h, i]]) == sorted(u)
+
+
+def test_union_intra_ties_are_flagged():
+    g = orc.Geometry(**dict(RAGGED, B=1))
+    p = _rand_p(g, 26)
+    v = np.arange(g.nb, dtype=np.float64)[None, None, :].repeat(2, axis=1) + 1.0
+    v[0, 0, 5] = v[0, 0, 6]                        # k = 2 cut between two equal scores
+    _, _, tie = orc.select_union(g, p, 0, [0.25, 0.25], intra=v, intra_params=[0.25, 0.25])
+    assert tie[0, 0].all()
