@@ -192,6 +192,52 @@ def effective_pairs(plan, idx, cnt) -> int:
     return video + text
 
 
+# Mask union timed beside the plain step: a window of one block on each side,
+# the blocks of the first latent frame as attention sink, and the 2% of key
+# blocks with the largest SICS (intra Top-K).
+UNION = dict(window=(1, 1), sink_frames=1, intra_mode=0, intra_density=0.02)
+
+
+def time_union_forward(bsa, w, plan, qd, kd, vd, out, dev, args, barrier):
+    """CUDA-event timing of bsa_forward_union over --steps steps."""
+    L = bsa.load()
+    u = bsa.mask_union(w.Hd, window=UNION["window"], sink_tokens=UNION["sink_frames"] * w.H * w.W,
+                       intra_mode=UNION["intra_mode"], intra_params=UNION["intra_density"])
+    kmax = plan.kmax_for_union(w.mode, w.params, u)
+    _, fwd_ws = plan.union_workspace_size(kmax, u)
+    ws = torch.empty(fwd_ws, dtype=torch.uint8, device=dev)
+    idx = torch.empty((w.B, w.Hd, plan.info.nb, kmax), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.B, w.Hd, plan.info.nb), dtype=torch.int32, device=dev)
+    params = bsa._params(w.params, w.Hd)
+    P = bsa._ptr
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        bsa._check(L.bsa_forward_union(plan._h, P(qd), P(kd), P(vd), w.mode, params, ctypes.byref(u),
+                                       kmax, P(out), P(idx), P(cnt), P(ws), ws.numel(), None,
+                                       bsa._stream(dev)))
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    plan.check_status()
+    pairs = effective_pairs(plan, idx, cnt)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    barrier()
+    plan.check_status()
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = 4.0 * pairs * w.D
+    return {"window": list(UNION["window"]), "sink_tokens": UNION["sink_frames"] * w.H * w.W,
+            "intra": f"top-k density {UNION['intra_density']} of K-block SICS",
+            "ms_per_step": round(ms, 4), "effective_tflop_per_step": round(flops / 1e12, 4),
+            "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+            "mean_list_len": round(float(cnt.float().mean()), 2), "selected_pairs": pairs}
+
+
 CANDIDATE_SHAPES = [(1, 8, 16), (4, 4, 8), (16, 1, 8), (2, 8, 8), (8, 2, 8)]
 
 
@@ -343,6 +389,9 @@ def run_ours(args, rank, world, local):
     del qb, kb, vb, ob
     phase_ms = fused if fused is not None else unfused
 
+    # ---- forward with the mask union (window, sink, intra blocks added)
+    union = time_union_forward(bsa, w, plan, qd, kd, vd, out, dev, args, barrier)
+
     # ---- scheme generation (aggregation evaluation over candidate blockings):
     # one launch evaluates three candidate schemes of Q; timed alone.
     scheme = time_scheme_generation(bsa, w, qd, dev, args, barrier)
@@ -476,6 +525,7 @@ def run_ours(args, rank, world, local):
                         "double-buffered device tensors)",
                 "serial": {"value": round(job_tflops(world, flops, e2e_serial_ms), 2),
                            "ms_per_step": round(e2e_serial_ms, 3)}},
+        "mask_union": dict(union, frac_of_peak=round(union["tflops"] / peak_tf, 4)),
         "scheme_generation": dict(scheme, share_of_attn=round(scheme["ms"] / phase_ms["attention"], 4),
                                   frac=round(scheme["achieved_gbs"] / hbm_gbs, 4),
                                   peak_gbs=hbm_gbs, bound="hbm"),

@@ -77,6 +77,10 @@ def load():
         "bsa_forward": [P, P, P, P, I, P, I, P, P, P, P, Z, P, P],
         "bsa_check_status": [P, P],
         "bsa_sics": [P, P, P, P],
+        "bsa_kmax_for_union": [P, I, P, P, ctypes.POINTER(I)],
+        "bsa_union_workspace_size": [P, I, P, ctypes.POINTER(Z), ctypes.POINTER(Z)],
+        "bsa_select_union": [P, P, P, I, P, P, P, I, P, P, P, P, Z, P],
+        "bsa_forward_union": [P, P, P, P, I, P, P, I, P, P, P, P, Z, P, P],
         "bsa_aggregation_scores": [P, I, P, P, P, P, P],
     }
     for name, args in sigs.items():
@@ -107,6 +111,24 @@ def _params(p, heads):
     if len(p) != heads:
         raise BsaError(1, f"expected {heads} per-head parameters, got {len(p)}")
     return arr
+
+
+class MaskUnion(ctypes.Structure):
+    """bsa_mask_union_t: window (left, right) in blocks, sink tokens, intra rule."""
+    _fields_ = [("window_left", ctypes.c_int), ("window_right", ctypes.c_int),
+                ("sink_tokens", ctypes.c_longlong), ("intra_mode", ctypes.c_int),
+                ("intra_param", ctypes.POINTER(ctypes.c_double))]
+
+
+def mask_union(heads, window=(-1, -1), sink_tokens=0, intra_mode=0, intra_params=None):
+    """A MaskUnion (kept alive with its per-head intra array)."""
+    u = MaskUnion(int(window[0]), int(window[1]), int(sink_tokens), int(intra_mode), None)
+    if intra_params is not None:
+        arr = _params(intra_params, heads) if not isinstance(intra_params, (int, float)) \
+            else _params([float(intra_params)] * heads, heads)
+        u._keep = arr
+        u.intra_param = ctypes.cast(arr, ctypes.POINTER(ctypes.c_double))
+    return u
 
 
 class Plan:
@@ -287,6 +309,57 @@ class Plan:
                                   _params(params, self.info.heads), kmax, _ptr(out), _ptr(idx),
                                   _ptr(cnt), _ptr(ws), ws.numel(), None, _stream(self.device)))
         return (out, idx, cnt) if return_lists else out
+
+    # --------------------------------------------------------- mask union
+    def kmax_for_union(self, mode, params, union) -> int:
+        k = ctypes.c_int()
+        _check(load().bsa_kmax_for_union(self._h, mode, _params(params, self.info.heads),
+                                         ctypes.byref(union) if union is not None else None,
+                                         ctypes.byref(k)))
+        return k.value
+
+    def union_workspace_size(self, kmax, union):
+        a, b = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(load().bsa_union_workspace_size(self._h, kmax,
+                                               ctypes.byref(union) if union is not None else None,
+                                               ctypes.byref(a), ctypes.byref(b)))
+        return a.value, b.value
+
+    def select_union(self, q_cent, k_cent, mode, params, union, intra_scores=None, kmax=None,
+                     scores=False):
+        """bsa_select_union: Top-K/Top-P lists united with window, sink and intra blocks."""
+        i = self.info
+        self._check_tensor(q_cent, self.cent_shape, torch.float32, "q_cent")
+        self._check_tensor(k_cent, self.cent_shape, torch.float32, "k_cent")
+        if intra_scores is not None:
+            self._check_tensor(intra_scores, (i.batch, i.heads, i.nb), torch.float32, "intra_scores")
+        kmax = kmax or self.kmax_for_union(mode, params, union)
+        idx, cnt = self._lists(kmax)
+        sc = self._new((i.batch, i.heads, i.nb, i.nb), torch.float32) if scores else None
+        sel_ws, _ = self.union_workspace_size(kmax, union)
+        ws = self._new((max(sel_ws, 1),), torch.uint8)
+        _check(load().bsa_select_union(self._h, _ptr(q_cent), _ptr(k_cent), mode,
+                                       _params(params, i.heads), ctypes.byref(union),
+                                       _ptr(intra_scores), kmax, _ptr(idx), _ptr(cnt), _ptr(sc),
+                                       _ptr(ws), ws.numel(), _stream(self.device)))
+        return (idx, cnt, sc) if scores else (idx, cnt)
+
+    def forward_union(self, q, k, v, mode, params, union, kmax=None, out=None, workspace=None,
+                      dev_status=None):
+        """bsa_forward_union: the whole path with the mask union; returns (o, idx, cnt)."""
+        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+            self._check_tensor(t, self.orig_shape, name=n)
+        kmax = kmax or self.kmax_for_union(mode, params, union)
+        idx, cnt = self._lists(kmax)
+        out = self._new(self.orig_shape) if out is None else out
+        _, fwd_ws = self.union_workspace_size(kmax, union)
+        ws = workspace if workspace is not None else self._new((max(fwd_ws, 1),), torch.uint8)
+        _check(load().bsa_forward_union(self._h, _ptr(q), _ptr(k), _ptr(v), mode,
+                                        _params(params, self.info.heads),
+                                        ctypes.byref(union) if union is not None else None, kmax,
+                                        _ptr(out), _ptr(idx), _ptr(cnt), _ptr(ws), ws.numel(),
+                                        _ptr(dev_status), _stream(self.device)))
+        return out, idx, cnt
 
     def check_status(self):
         """Synchronise the current stream and raise if a kernel recorded an error."""

@@ -152,12 +152,75 @@ bsa_status make_orig_maps(CUtensorMap* video, CUtensorMap* text, const void* x, 
   return BSA_OK;
 }
 
+// Host copy of a validated mask union (window, sink, intra selection).
+struct UnionOpts {
+  int win_left = -1, win_right = -1;
+  long long sink_tokens = 0;
+  bool intra = false;
+  int intra_mode = 0;
+  double intra_param[BSA_MAX_HEADS] = {};   // k (held in a double) or tau per head; <= 0 = none
+};
+
+size_t bits_bytes(const bsa_plan_s* p) {
+  return (size_t)p->g.B * p->g.Hd * ((p->g.nb + 31) / 32) * sizeof(uint32_t);
+}
+size_t sics_bytes(const bsa_plan_s* p) { return (size_t)p->g.B * p->g.Hd * p->g.nb * sizeof(float); }
+
+// Validates `u` (NULL = no union) and returns the number of video key blocks
+// it can add to one list on top of the inter selection.
+bsa_status check_union(const bsa_plan_s* p, const bsa_mask_union_t* u, UnionOpts* o, int* extra) {
+  *o = UnionOpts();
+  *extra = 0;
+  if (u == nullptr) return BSA_OK;
+  const int nb = p->g.nb;
+  o->win_left = u->window_left;
+  o->win_right = u->window_right;
+  o->sink_tokens = u->sink_tokens;
+  if (u->sink_tokens < 0) return fail(BSA_ERR_INVALID_ARG, "sink_tokens must be >= 0");
+  long long add = 0;
+  if (u->window_left >= 0 || u->window_right >= 0)
+    add += (u->window_left < 0 || u->window_right < 0)
+               ? nb : (long long)u->window_left + u->window_right + 1;
+  if (u->sink_tokens > 0) {
+    const Geo& g = p->g;
+    for (int j = 0; j < nb; ++j) {
+      const int xb = j % g.nbx, yb = (j / g.nbx) % g.nby, tb = j / (g.nbx * g.nby);
+      const long long first = ((long long)tb * g.bf * g.H + (long long)yb * g.br) * g.W +
+                              (long long)xb * g.bc;
+      if (first < u->sink_tokens) ++add;
+    }
+  }
+  if (u->intra_param != nullptr) {
+    if (u->intra_mode != BSA_TOPK && u->intra_mode != BSA_TOPP)
+      return fail(BSA_ERR_INVALID_ARG, "bad intra mode %d", (int)u->intra_mode);
+    o->intra_mode = (int)u->intra_mode;
+    int kmax_intra = 0;
+    for (int h = 0; h < p->g.Hd; ++h) {
+      const double v = u->intra_param[h];
+      if (!(v >= 0.0 && v <= 1.0))
+        return fail(BSA_ERR_INVALID_ARG, "intra %s of head %d is %g, must be in [0, 1]",
+                    u->intra_mode == BSA_TOPK ? "density" : "tau", h, v);
+      if (v > 0.0) {
+        o->intra = true;
+        o->intra_param[h] = u->intra_mode == BSA_TOPK ? (double)k_for_density(v, nb) : v;
+        const int k = u->intra_mode == BSA_TOPK ? k_for_density(v, nb) : nb;
+        if (k > kmax_intra) kmax_intra = k;
+      }
+    }
+    add += kmax_intra;
+  }
+  *extra = (int)(add < nb ? add : nb);
+  return BSA_OK;
+}
+
 bsa_status run_select(const bsa_plan_s* p, const float* qc, const float* kc, bsa_select_mode mode,
                       const double* param, int kmax, int32_t* idx, int32_t* cnt, float* scores,
-                      cudaStream_t st) {
+                      cudaStream_t st, const UnionOpts* uo = nullptr, const float* intra_scores = nullptr,
+                      uint32_t* bits = nullptr) {
   int need = 0;
   bsa_status s = check_params(p, mode, param, &need);
   if (s != BSA_OK) return s;
+  // (union callers check kmax against the union's bound themselves)
   if (kmax < need) return fail(BSA_ERR_INVALID_ARG, "kmax %d is below the %d entries a list can need", kmax, need);
   if (p->g.nb == 0) return BSA_OK;
   if (!qc || !kc || !idx || !cnt) return fail(BSA_ERR_INVALID_ARG, "NULL centroid or list pointer");
@@ -169,6 +232,24 @@ bsa_status run_select(const bsa_plan_s* p, const float* qc, const float* kc, bsa
   a.scale = (float)(1.0 / std::sqrt((double)p->g.D));
   for (int h = 0; h < p->g.Hd; ++h)
     a.param[h] = mode == BSA_TOPK ? (double)k_for_density(param[h], p->g.nb) : param[h];
+  a.win_left = a.win_right = -1;
+  if (uo != nullptr) {
+    a.win_left = uo->win_left;
+    a.win_right = uo->win_right;
+    a.sink_tokens = uo->sink_tokens;
+    if (uo->intra) {
+      if (!intra_scores || !bits) return fail(BSA_ERR_INVALID_ARG, "intra selection needs intra scores");
+      bsa::IntraArgs ia;
+      std::memset(&ia, 0, sizeof(ia));
+      ia.scores = intra_scores;
+      ia.bits = bits;
+      ia.mode = uo->intra_mode;
+      for (int h = 0; h < p->g.Hd; ++h) ia.param[h] = uo->intra_param[h];
+      cudaError_t e = bsa::launch_intra_select(p->g, ia, st);
+      if (e != cudaSuccess) return cuda_fail(e, "intra select kernel");
+      a.intra_bits = bits;
+    }
+  }
   cudaError_t e = bsa::launch_select(p->g, a, st);
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "select kernel");
 }
@@ -204,12 +285,15 @@ bsa_status run_attention(const bsa_plan_s* p, const void* q, const void* k, cons
 }
 
 bsa_status run_centroids(const bsa_plan_s* p, const void* q, const void* k, float* qc, float* kc,
-                         cudaStream_t st) {
+                         cudaStream_t st, float* k_sics = nullptr) {
   // Only the requested tensors are read.
   bsa::GatherArgs ga;
   std::memset(&ga, 0, sizeof(ga));
   if (qc) { ga.src[ga.ntensors] = q; ga.cent[ga.ntensors] = qc; ++ga.ntensors; }
-  if (kc) { ga.src[ga.ntensors] = k; ga.cent[ga.ntensors] = kc; ++ga.ntensors; }
+  if (kc) {
+    ga.src[ga.ntensors] = k; ga.cent[ga.ntensors] = kc; ga.sics[ga.ntensors] = k_sics;
+    ++ga.ntensors;
+  }
   if (ga.ntensors == 0 || p->g.nb == 0) return BSA_OK;
   cudaError_t e = bsa::launch_pool_orig(p->g, p->dtype == BSA_BF16, ga, st);
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "centroid kernel");
@@ -261,11 +345,88 @@ bsa_status run_attention_orig(const bsa_plan_s* p, const void* q, const void* k,
 bsa_status run_forward_fused(const bsa_plan_s* p, const void* q, const void* k, const void* v,
                              bsa_select_mode mode, const double* param, int kmax, void* o,
                              int32_t* idx, int32_t* cnt, float* qc, float* kc,
-                             int32_t* dev_status, cudaStream_t st) {
-  bsa_status s = run_centroids(p, q, k, qc, kc, st);
+                             int32_t* dev_status, cudaStream_t st, const UnionOpts* uo = nullptr,
+                             float* k_sics = nullptr, uint32_t* bits = nullptr) {
+  bsa_status s = run_centroids(p, q, k, qc, kc, st, k_sics);
   if (s != BSA_OK) return s;
-  if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st)) != BSA_OK) return s;
+  if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st, uo, k_sics, bits)) != BSA_OK)
+    return s;
   return run_attention_orig(p, q, k, v, idx, cnt, kmax, o, dev_status, st);
+}
+
+// kmax a list can need under the union: the inter bound plus the blocks the
+// union can add, at most every video block, plus the text blocks.
+bsa_status union_kmax(const bsa_plan_s* p, bsa_select_mode mode, const double* param,
+                      const bsa_mask_union_t* u, int* kmax) {
+  int need = 0, extra = 0;
+  bsa_status s = check_params(p, mode, param, &need);
+  if (s != BSA_OK) return s;
+  UnionOpts uo;
+  if ((s = check_union(p, u, &uo, &extra)) != BSA_OK) return s;
+  const int video = need - p->g.nb_text + extra;
+  *kmax = (video < p->g.nb ? video : p->g.nb) + p->g.nb_text;
+  return BSA_OK;
+}
+
+bsa_status forward_impl(bsa_plan_t p, const void* q, const void* k, const void* v,
+                        bsa_select_mode mode, const double* param, const bsa_mask_union_t* u,
+                        int kmax, void* o, int32_t* idx_out, int32_t* cnt_out, void* ws,
+                        size_t ws_bytes, int32_t* dev_status, void* stream) {
+  bsa_status s = check_plan(p);
+  if (s != BSA_OK) return s;
+  int need = 0;
+  if ((s = union_kmax(p, mode, param, u, &need)) != BSA_OK) return s;
+  if (kmax < need) return fail(BSA_ERR_INVALID_ARG, "kmax %d is below the %d entries a list can need", kmax, need);
+  UnionOpts uo;
+  int extra = 0;
+  if ((s = check_union(p, u, &uo, &extra)) != BSA_OK) return s;
+  if (!q || !k || !v || !o) return fail(BSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  size_t base_ws = 0;
+  bsa_workspace_size(p, kmax, nullptr, &base_ws);
+  const size_t need_ws = base_ws + (uo.intra ? round256(bits_bytes(p)) + round256(sics_bytes(p)) : 0);
+  if (ws == nullptr || ws_bytes < need_ws)
+    return fail(BSA_ERR_WORKSPACE, "forward needs %zu bytes of workspace, got %zu", need_ws, ws_bytes);
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(BSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  char* w = reinterpret_cast<char*>(ws);
+  const size_t tb = p->attn_path == 1 ? 0 : round256(blk_bytes(p)), cb = round256(cent_bytes(p));
+  void* q_blk = w; w += tb;
+  void* k_blk = w; w += tb;
+  void* v_blk = w; w += tb;
+  void* o_blk = w; w += tb;
+  float* qc = reinterpret_cast<float*>(w); w += cb;
+  float* kc = reinterpret_cast<float*>(w); w += cb;
+  int32_t* idx = reinterpret_cast<int32_t*>(w);
+  w += round256((size_t)p->g.B * p->g.Hd * p->g.nb * kmax * sizeof(int32_t));
+  int32_t* cnt = reinterpret_cast<int32_t*>(w);
+  w += round256((size_t)p->g.B * p->g.Hd * p->g.nb * sizeof(int32_t));
+  float* k_sics = nullptr;
+  uint32_t* bits = nullptr;
+  if (uo.intra) {
+    k_sics = reinterpret_cast<float*>(w); w += round256(sics_bytes(p));
+    bits = reinterpret_cast<uint32_t*>(w);
+  }
+  if (idx_out) idx = idx_out;
+  if (cnt_out) cnt = cnt_out;
+  cudaStream_t st = (cudaStream_t)stream;
+  const UnionOpts* up = u ? &uo : nullptr;
+  if (p->attn_path == 1)
+    return run_forward_fused(p, q, k, v, mode, param, kmax, o, idx, cnt, qc, kc, dev_status, st, up,
+                             k_sics, bits);
+  bsa::GatherArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.src[0] = q; a.src[1] = k; a.src[2] = v;
+  a.dst[0] = q_blk; a.dst[1] = k_blk; a.dst[2] = v_blk;
+  a.cent[0] = qc; a.cent[1] = kc;
+  a.sics[1] = k_sics;
+  a.ntensors = 3;
+  cudaError_t e = bsa::launch_permute(p->g, p->dtype == BSA_BF16, a, st);
+  if (e != cudaSuccess) return cuda_fail(e, "permute kernel");
+  if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st, up, k_sics, bits)) != BSA_OK)
+    return s;
+  if ((s = run_attention(p, q_blk, k_blk, v_blk, idx, cnt, kmax, o_blk, dev_status, st)) != BSA_OK) return s;
+  return bsa_unpermute(p, o_blk, o, stream);
 }
 
 }  // namespace
@@ -484,41 +645,64 @@ bsa_status bsa_forward(bsa_plan_t p, const void* q, const void* k, const void* v
                        bsa_select_mode mode, const double* param, int kmax, void* o,
                        int32_t* idx_out, int32_t* cnt_out, void* ws, size_t ws_bytes,
                        int32_t* dev_status, void* stream) {
+  return forward_impl(p, q, k, v, mode, param, nullptr, kmax, o, idx_out, cnt_out, ws, ws_bytes,
+                      dev_status, stream);
+}
+
+bsa_status bsa_kmax_for_union(bsa_plan_t p, bsa_select_mode mode, const double* param,
+                              const bsa_mask_union_t* u, int* kmax) {
+  if (p == nullptr || kmax == nullptr) return fail(BSA_ERR_INVALID_ARG, "NULL plan or output");
+  return union_kmax(p, mode, param, u, kmax);
+}
+
+bsa_status bsa_union_workspace_size(bsa_plan_t p, int kmax, const bsa_mask_union_t* u,
+                                    size_t* select_ws, size_t* forward_ws) {
+  if (p == nullptr) return fail(BSA_ERR_INVALID_ARG, "plan is NULL");
+  UnionOpts uo;
+  int extra = 0;
+  bsa_status s = check_union(p, u, &uo, &extra);
+  if (s != BSA_OK) return s;
+  size_t base = 0;
+  if ((s = bsa_workspace_size(p, kmax, nullptr, &base)) != BSA_OK) return s;
+  const size_t add_sel = uo.intra ? round256(bits_bytes(p)) : 0;
+  const size_t add_fwd = uo.intra ? round256(bits_bytes(p)) + round256(sics_bytes(p)) : 0;
+  if (select_ws) *select_ws = add_sel;
+  if (forward_ws) *forward_ws = base + add_fwd;
+  return BSA_OK;
+}
+
+bsa_status bsa_select_union(bsa_plan_t p, const float* q_cent, const float* k_cent,
+                            bsa_select_mode mode, const double* param, const bsa_mask_union_t* u,
+                            const float* intra_scores, int kmax, int32_t* idx, int32_t* cnt,
+                            float* scores, void* ws, size_t ws_bytes, void* stream) {
   bsa_status s = check_plan(p);
   if (s != BSA_OK) return s;
   int need = 0;
-  if ((s = check_params(p, mode, param, &need)) != BSA_OK) return s;
+  if ((s = union_kmax(p, mode, param, u, &need)) != BSA_OK) return s;
   if (kmax < need) return fail(BSA_ERR_INVALID_ARG, "kmax %d is below the %d entries a list can need", kmax, need);
-  if (!q || !k || !v || !o) return fail(BSA_ERR_INVALID_ARG, "NULL tensor pointer");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
-    return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
-  size_t need_ws = 0;
-  bsa_workspace_size(p, kmax, nullptr, &need_ws);
-  if (ws == nullptr || ws_bytes < need_ws)
-    return fail(BSA_ERR_WORKSPACE, "forward needs %zu bytes of workspace, got %zu", need_ws, ws_bytes);
-  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(BSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
-  char* w = reinterpret_cast<char*>(ws);
-  const size_t tb = p->attn_path == 1 ? 0 : round256(blk_bytes(p)), cb = round256(cent_bytes(p));
-  void* q_blk = w; w += tb;
-  void* k_blk = w; w += tb;
-  void* v_blk = w; w += tb;
-  void* o_blk = w; w += tb;
-  float* qc = reinterpret_cast<float*>(w); w += cb;
-  float* kc = reinterpret_cast<float*>(w); w += cb;
-  int32_t* idx = reinterpret_cast<int32_t*>(w);
-  w += round256((size_t)p->g.B * p->g.Hd * p->g.nb * kmax * sizeof(int32_t));
-  int32_t* cnt = reinterpret_cast<int32_t*>(w);
-  if (idx_out) idx = idx_out;
-  if (cnt_out) cnt = cnt_out;
-  cudaStream_t st = (cudaStream_t)stream;
-  if (p->attn_path == 1)
-    return run_forward_fused(p, q, k, v, mode, param, kmax, o, idx, cnt, qc, kc, dev_status, st);
-  if ((s = bsa_permute_qkv(p, q, k, v, q_blk, k_blk, v_blk, qc, kc, stream)) != BSA_OK) return s;
-  if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st)) != BSA_OK) return s;
-  if ((s = run_attention(p, q_blk, k_blk, v_blk, idx, cnt, kmax, o_blk, dev_status, st)) != BSA_OK) return s;
-  return bsa_unpermute(p, o_blk, o, stream);
+  UnionOpts uo;
+  int extra = 0;
+  if ((s = check_union(p, u, &uo, &extra)) != BSA_OK) return s;
+  uint32_t* bits = nullptr;
+  if (uo.intra) {
+    if (intra_scores == nullptr) return fail(BSA_ERR_INVALID_ARG, "intra selection needs intra_scores");
+    if (ws == nullptr || ws_bytes < bits_bytes(p))
+      return fail(BSA_ERR_WORKSPACE, "union selection needs %zu bytes of workspace, got %zu",
+                  round256(bits_bytes(p)), ws_bytes);
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(BSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    bits = reinterpret_cast<uint32_t*>(ws);
+  }
+  return run_select(p, q_cent, k_cent, mode, param, kmax, idx, cnt, scores, (cudaStream_t)stream,
+                    &uo, intra_scores, bits);
 }
 
+bsa_status bsa_forward_union(bsa_plan_t p, const void* q, const void* k, const void* v,
+                             bsa_select_mode mode, const double* param, const bsa_mask_union_t* u,
+                             int kmax, void* o, int32_t* idx_out, int32_t* cnt_out, void* ws,
+                             size_t ws_bytes, int32_t* dev_status, void* stream) {
+  return forward_impl(p, q, k, v, mode, param, u, kmax, o, idx_out, cnt_out, ws, ws_bytes,
+                      dev_status, stream);
+}
 bsa_status bsa_sics(bsa_plan_t p, const void* x, float* sics, void* stream) {
   bsa_plan_t plans[1] = {p};
   float* outs[1] = {sics};

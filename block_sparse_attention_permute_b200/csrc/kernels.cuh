@@ -36,6 +36,18 @@ struct SelectArgs {
   int mode;          // 0 top-k, 1 top-p
   float scale;       // 1/sqrt(D) rounded to fp32
   double param[BSA_MAX_HEADS];  // k (held in a double) or tau, per head
+  // Mask union (video key blocks added to every list of a head):
+  int win_left, win_right;      // j in [i - left, i + right]; < 0 = unbounded; both < 0 = none
+  long long sink_tokens;        // blocks holding any of the first sink_tokens tokens
+  const uint32_t* intra_bits;   // [B, Hd, nbw] selected key blocks, or null
+};
+
+// Selection on per-key-block intra scores (one warp per (b, h)).
+struct IntraArgs {
+  const float* scores;          // [B, Hd, nb]
+  uint32_t* bits;               // [B, Hd, nbw], nbw = ceil(nb / 32)
+  int mode;                     // 0 top-k, 1 top-p
+  double param[BSA_MAX_HEADS];  // k (held in a double) or tau per head; <= 0 = none
 };
 
 struct AttnArgs {
@@ -67,6 +79,7 @@ cudaError_t launch_sics_schemes(const SchemeArgs& a, bool is_bf16, cudaStream_t 
 // select.cu
 size_t select_smem_bytes(int nb, int D);
 cudaError_t launch_select(const Geo& g, const SelectArgs& a, cudaStream_t st);
+cudaError_t launch_intra_select(const Geo& g, const IntraArgs& a, cudaStream_t st);
 // attn.cu
 size_t attn_tc_smem_bytes(int D);
 cudaError_t launch_attn_simt(const Geo& g, bool is_bf16, const AttnArgs& a, cudaStream_t st);

@@ -48,12 +48,23 @@ __device__ __forceinline__ int warp_count(bool pred) {
   return __popc(__ballot_sync(0xffffffffu, pred));
 }
 
-// sum over j with key(s_j) >= cand of expf(s_j - m), in fp64, fixed order.
-__device__ double mass_at_least(const float* row, int nb, float m, uint32_t cand, int lane) {
+// Weight of a score in the Top-P mass: expf(s - m) for the softmax of the
+// inter-block scores, the score itself for intra scores.
+struct SoftmaxWeight {
+  float m;
+  __device__ __forceinline__ double operator()(float s) const { return (double)expf(s - m); }
+};
+struct PlainWeight {
+  __device__ __forceinline__ double operator()(float s) const { return (double)s; }
+};
+
+// sum over j with key(s_j) >= cand of wt(s_j), in fp64, fixed order.
+template <class Wt>
+__device__ double mass_at_least(const float* row, int nb, Wt wt, uint32_t cand, int lane) {
   double acc = 0.0;
   for (int j = lane; j < nb; j += 32) {
     const float s = row[j];
-    if (order_key(s) >= cand) acc += (double)expf(s - m);
+    if (order_key(s) >= cand) acc += wt(s);
   }
   return warp_sum_uniform(acc);
 }
@@ -82,6 +93,78 @@ __device__ __forceinline__ uint32_t kth_largest_key(const uint32_t (&kr)[kKeysPe
     if (c >= k) T = cand;
   }
   return T;
+}
+
+// Threshold of the Top-K / Top-P rule over one row of nb scores: every entry
+// with order key > T is taken, plus the first `need` (ascending j) of those
+// with key == T.  Top-K: param = k.  Top-P: param = tau, `total` = the sum of
+// all weights; the shortest descending prefix whose weight reaches
+// tau * total (at least one entry).
+template <class Wt>
+__device__ __forceinline__ void rule_threshold(const float* row, int nb, int mode, double param,
+                                               double total, Wt wt, int lane, uint32_t* T_out,
+                                               int* need_out) {
+  uint32_t T = 0;
+  int need = 0;
+  const double target = param * total;
+  if (mode != 0 && !(target > 0.0)) {   // every prefix reaches 0: one entry
+    mode = 0;
+    param = 1.0;
+  }
+  if (mode == 0) {
+    const int k = (int)param;
+    if (nb <= 32 * kKeysPerLane) {
+      // order_key of any float is nonzero and every candidate threshold is
+      // nonzero, so the 0 used for missing entries never counts
+      uint32_t kr[kKeysPerLane];
+#pragma unroll
+      for (int e = 0; e < kKeysPerLane; ++e) {
+        const int j = lane + 32 * e;
+        kr[e] = j < nb ? order_key(row[j]) : 0u;
+      }
+      T = kth_largest_key(kr, k);
+      int c = 0;
+#pragma unroll
+      for (int e = 0; e < kKeysPerLane; ++e) c += kr[e] > T ? 1 : 0;
+      need = k - __reduce_add_sync(0xffffffffu, c);
+    } else {
+      for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = T | (1u << bit);
+        if (count_at_least(row, nb, cand, lane) >= k) T = cand;
+      }
+      const int n_gt = (T == 0xffffffffu) ? 0 : count_at_least(row, nb, T + 1, lane);
+      need = k - n_gt;
+    }
+  } else {
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      if (mass_at_least(row, nb, wt, cand, lane) >= target) T = cand;
+    }
+    double acc = (T == 0xffffffffu) ? 0.0 : mass_at_least(row, nb, wt, T + 1, lane);
+    int n_eq = 0;
+    float s_eq = 0.f;
+    for (int j = lane; j < nb; j += 32)
+      if (order_key(row[j]) == T) { ++n_eq; s_eq = row[j]; }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      n_eq += __shfl_xor_sync(0xffffffffu, n_eq, off);
+      s_eq = fmaxf(s_eq, __shfl_xor_sync(0xffffffffu, s_eq, off));
+    }
+    const double e_eq = wt(s_eq);
+    while (acc < target && need < n_eq) {
+      acc += e_eq;
+      ++need;
+    }
+    if (need == 0) need = 1;
+  }
+  *T_out = T;
+  *need_out = need;
+}
+
+// First token (in the original order) of video block j: its corner.
+__device__ __forceinline__ long long block_first_token(const Geo& g, int j) {
+  const int xb = j % g.nbx, yb = (j / g.nbx) % g.nby, tb = j / (g.nbx * g.nby);
+  return ((long long)tb * g.bf * g.H + (long long)yb * g.br) * g.W + (long long)xb * g.bc;
 }
 
 template <int D>
@@ -158,7 +241,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, SelectArgs a
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     // The normaliser is needed only for the score output and for Top-P
     // (Top-K depends on the order of the scores alone).
-    const double Z = (a.scores != nullptr || a.mode != 0) ? mass_at_least(row, nb, m, 0u, lane) : 1.0;
+    const double Z = (a.scores != nullptr || a.mode != 0)
+                         ? mass_at_least(row, nb, SoftmaxWeight{m}, 0u, lane) : 1.0;
 
     if (a.scores != nullptr) {
       float* out = a.scores + (bh * nb + i) * nb;
@@ -167,65 +251,29 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, SelectArgs a
 
     uint32_t T = 0;
     int need = 0;  // how many of the scores equal to the threshold to take
-    if (a.mode == 0) {
-      const int k = (int)a.param[h];
-      if (nb <= 32 * kKeysPerLane) {
-        // order_key of any float is nonzero and every candidate threshold is
-        // nonzero, so the 0 used for missing entries never counts
-        uint32_t kr[kKeysPerLane];
-#pragma unroll
-        for (int e = 0; e < kKeysPerLane; ++e) {
-          const int j = lane + 32 * e;
-          kr[e] = j < nb ? order_key(row[j]) : 0u;
-        }
-        T = kth_largest_key(kr, k);
-        int c = 0;
-#pragma unroll
-        for (int e = 0; e < kKeysPerLane; ++e) c += kr[e] > T ? 1 : 0;
-        need = k - __reduce_add_sync(0xffffffffu, c);
-      } else {
-        for (int bit = 31; bit >= 0; --bit) {
-          const uint32_t cand = T | (1u << bit);
-          if (count_at_least(row, nb, cand, lane) >= k) T = cand;
-        }
-        const int n_gt = (T == 0xffffffffu) ? 0 : count_at_least(row, nb, T + 1, lane);
-        need = k - n_gt;
-      }
-    } else {
-      const double target = a.param[h] * Z;
-      for (int bit = 31; bit >= 0; --bit) {
-        const uint32_t cand = T | (1u << bit);
-        if (mass_at_least(row, nb, m, cand, lane) >= target) T = cand;
-      }
-      double acc = (T == 0xffffffffu) ? 0.0 : mass_at_least(row, nb, m, T + 1, lane);
-      int n_eq = 0;
-      float s_eq = 0.f;
-      for (int j = lane; j < nb; j += 32)
-        if (order_key(row[j]) == T) { ++n_eq; s_eq = row[j]; }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        n_eq += __shfl_xor_sync(0xffffffffu, n_eq, off);
-        s_eq = fmaxf(s_eq, __shfl_xor_sync(0xffffffffu, s_eq, off));
-      }
-      const double e_eq = (double)expf(s_eq - m);
-      while (acc < target && need < n_eq) {
-        acc += e_eq;
-        ++need;
-      }
-      if (need == 0) need = 1;
-    }
+    rule_threshold(row, nb, a.mode, a.param[h], Z, SoftmaxWeight{m}, lane, &T, &need);
 
-    // Ascending compaction of {key > T} plus the first `need` of {key == T}.
+    // Ascending compaction of {key > T} plus the first `need` of {key == T},
+    // united with the window, sink and intra blocks.
     int32_t* out = a.idx + (bh * nb + i) * a.kmax;
     int written = 0, eq_seen = 0;
     const uint32_t lt_mask = (1u << lane) - 1u;
+    const bool window = a.win_left >= 0 || a.win_right >= 0;
+    const long long w_lo = a.win_left < 0 ? 0 : (long long)i - a.win_left;
+    const long long w_hi = a.win_right < 0 ? nb : (long long)i + a.win_right;
+    const uint32_t* ibits = a.intra_bits ? a.intra_bits + bh * ((nb + 31) / 32) : nullptr;
     for (int j0 = 0; j0 < nb; j0 += 32) {
       const int j = j0 + lane;
       const uint32_t key = j < nb ? order_key(row[j]) : 0u;
       const bool gt = j < nb && key > T;
       const bool eq = j < nb && key == T;
       const uint32_t eq_bal = __ballot_sync(0xffffffffu, eq);
-      const bool take = gt || (eq && eq_seen + __popc(eq_bal & lt_mask) < need);
+      bool take = gt || (eq && eq_seen + __popc(eq_bal & lt_mask) < need);
+      if (j < nb) {
+        take = take || (window && j >= w_lo && j <= w_hi);
+        take = take || (a.sink_tokens > 0 && block_first_token(g, j) < a.sink_tokens);
+        take = take || (ibits != nullptr && ((ibits[j >> 5] >> (j & 31)) & 1u));
+      }
       const uint32_t sel_bal = __ballot_sync(0xffffffffu, take);
       if (take) out[written + __popc(sel_bal & lt_mask)] = j;
       written += __popc(sel_bal);
@@ -234,6 +282,49 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, SelectArgs a
     for (int t = lane; t < g.nb_text; t += 32) out[written + t] = nb + t;
     if (lane == 0) a.cnt[bh * nb + i] = written + g.nb_text;
   }
+}
+
+// Intra selection (SPADE §3.3: intra scores, one per block, filtered by the
+// intra-top value and broadcast to every query block): per (b, h) the same
+// Top-K / Top-P rule on the intra scores, with a score's own value as its
+// Top-P weight; the selected key blocks are written as a bit set.
+constexpr int kIntraWarps = 4;
+
+__global__ void __launch_bounds__(kIntraWarps * 32) intra_select_kernel(Geo g, IntraArgs a) {
+  const int bh = blockIdx.x * kIntraWarps + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (bh >= g.B * g.Hd) return;
+  const int nb = g.nb, nbw = (nb + 31) / 32, h = bh % g.Hd;
+  const float* row = a.scores + (long long)bh * nb;
+  uint32_t* bits = a.bits + (long long)bh * nbw;
+  const double prm = a.param[h];
+  if (!(prm > 0.0)) {
+    for (int w = lane; w < nbw; w += 32) bits[w] = 0u;
+    return;
+  }
+  const double total = a.mode != 0 ? mass_at_least(row, nb, PlainWeight{}, 0u, lane) : 0.0;
+  uint32_t T = 0;
+  int need = 0;
+  rule_threshold(row, nb, a.mode, prm, total, PlainWeight{}, lane, &T, &need);
+  int eq_seen = 0;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int j0 = 0; j0 < nb; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t key = j < nb ? order_key(row[j]) : 0u;
+    const bool gt = j < nb && key > T;
+    const bool eq = j < nb && key == T;
+    const uint32_t eq_bal = __ballot_sync(0xffffffffu, eq);
+    const bool take = gt || (eq && eq_seen + __popc(eq_bal & lt_mask) < need);
+    const uint32_t sel_bal = __ballot_sync(0xffffffffu, take);
+    if (lane == 0) bits[j0 >> 5] = sel_bal;
+    eq_seen += __popc(eq_bal);
+  }
+}
+
+cudaError_t launch_intra_select(const Geo& g, const IntraArgs& a, cudaStream_t st) {
+  const int BH = g.B * g.Hd;
+  if (BH == 0 || g.nb == 0) return cudaSuccess;
+  intra_select_kernel<<<(BH + kIntraWarps - 1) / kIntraWarps, kIntraWarps * 32, 0, st>>>(g, a);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_select(const Geo& g, const SelectArgs& a, cudaStream_t st) {

@@ -279,6 +279,81 @@ bsa_status bsa_forward(bsa_plan_t plan, const void* q, const void* k,
                        int32_t* idx_out, int32_t* cnt_out, void* ws,
                        size_t ws_bytes, int32_t* dev_status, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Mask union (SPADE §3.3: "intra scores are broadcast and OR-combined with
+ * inter scores.  The result is united with local-window and attention-sink
+ * masks to form a binary attention mask"; §3.2: each head's sparsity-ratio
+ * scheme has a local-window length, an intra-top value and an inter-top
+ * value; §3.1: attention-sink length).  Every entry is a whole video key
+ * block added to the lists of a head, so the attention kernels are unchanged.
+ * For video query block i of head h the list is the ascending union of
+ *   inter   the Top-K / Top-P selection of bsa_select;
+ *   window  key blocks j with i - window_left <= j <= i + window_right, a
+ *           sliding window over the block sequence in block units, like the
+ *           (left, right) window_size of LongLive's attention ("How to
+ *           Configure Local Attention Size for Long Video Generation in
+ *           LongLive"); a negative side is unbounded, and window_left < 0
+ *           together with window_right < 0 adds nothing;
+ *   sink    the key blocks that hold any of the first sink_tokens tokens of
+ *           the original order (0 = none);
+ *   intra   when intra_param is not NULL and intra_param[h] > 0: the key
+ *           blocks the intra_mode rule selects from one intra score per key
+ *           block, broadcast to every query block of the head.  Top-K keeps
+ *           ceil(intra_param[h] * nb - 1e-9) blocks with the largest scores;
+ *           Top-P keeps the shortest descending prefix whose score sum
+ *           reaches intra_param[h] * (sum of the head's scores).  Equal
+ *           scores are ordered by ascending block id;
+ * followed by the nb_text text key blocks.  Text query blocks stay dense. */
+typedef struct {
+  int window_left;               /* blocks before i; < 0 = unbounded         */
+  int window_right;              /* blocks after i;  < 0 = unbounded         */
+  long long sink_tokens;         /* >= 0                                      */
+  bsa_select_mode intra_mode;    /* rule applied to the intra scores          */
+  const double* intra_param;     /* host [Hd] in [0, 1], or NULL (no intra)   */
+} bsa_mask_union_t;
+
+/* bsa_kmax_for_union — list width that suffices under `u` (NULL = plain
+ * selection): the inter bound plus what the window, sink and intra parts can
+ * add, at most nb, plus nb_text. */
+bsa_status bsa_kmax_for_union(bsa_plan_t plan, bsa_select_mode mode,
+                              const double* param_per_head,
+                              const bsa_mask_union_t* u, int* kmax);
+
+/* bsa_union_workspace_size — device workspace (256-byte aligned) of
+ * bsa_select_union (select_ws: the intra bit sets, 0 without intra) and of
+ * bsa_forward_union (forward_ws: bsa_forward's plus, with intra, the SICS of
+ * the K blocks and the bit sets). */
+bsa_status bsa_union_workspace_size(bsa_plan_t plan, int kmax,
+                                    const bsa_mask_union_t* u,
+                                    size_t* select_ws, size_t* forward_ws);
+
+/* bsa_select_union — bsa_select_centroids with the mask union.
+ *   intra_scores  [B, Hd, nb] float device, one score per key block
+ *                 (required when u->intra_param is set; e.g. bsa_sics of K)
+ *   ws, ws_bytes  at least select_ws bytes (may be NULL / 0 without intra)
+ * Other arguments as bsa_select_centroids; kmax >= bsa_kmax_for_union. */
+bsa_status bsa_select_union(bsa_plan_t plan, const float* q_cent,
+                            const float* k_cent, bsa_select_mode mode,
+                            const double* param_per_head,
+                            const bsa_mask_union_t* u,
+                            const float* intra_scores, int kmax,
+                            int32_t* idx, int32_t* cnt, float* scores,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* bsa_forward_union — bsa_forward with the mask union; the intra scores are
+ * the SICS of the K blocks (SPADE §3.2 Eq. (4)), computed in the centroid
+ * pass that reads K anyway (SPADE §3.3 (1): layout transform, summarization
+ * and intra-estimation fused).  ws_bytes >= forward_ws of
+ * bsa_union_workspace_size; kmax >= bsa_kmax_for_union.  u = NULL is
+ * bsa_forward. */
+bsa_status bsa_forward_union(bsa_plan_t plan, const void* q, const void* k,
+                             const void* v, bsa_select_mode mode,
+                             const double* param_per_head,
+                             const bsa_mask_union_t* u, int kmax, void* o,
+                             int32_t* idx_out, int32_t* cnt_out, void* ws,
+                             size_t ws_bytes, int32_t* dev_status,
+                             void* stream);
+
 /* bsa_check_status — synchronise `stream`, read and clear the plan-owned
  * status word; returns BSA_OK or the recorded error. */
 bsa_status bsa_check_status(bsa_plan_t plan, void* stream);

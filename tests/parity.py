@@ -143,3 +143,98 @@ def check_sics(g, gpu, ref, what=""):
     worst = float((err / tol).max()) if err.size else 0.0
     assert worst <= 1.0, f"{what}: SICS error {float(err.max()):.3e} above its bound (x{worst:.2f})"
     return (float(err.max()) if err.size else 0.0), worst
+
+
+# ------------------------------------------------------------ mask union --
+def union_extras(g, window, sink_tokens, intra_sets):
+    """Per (b, h, i): the set of video key blocks the window, sink and intra
+    parts add (intra_sets[b][h] = set of key blocks or empty)."""
+    wl, wr = window
+    sink = set()
+    for j in range(g.nb):
+        tb, yb, xb = j // (g.nby * g.nbx), (j // g.nbx) % g.nby, j % g.nbx
+        first = (tb * g.bf * g.H + yb * g.br) * g.W + xb * g.bc
+        if first < sink_tokens:
+            sink.add(j)
+    out = {}
+    for b in range(g.B):
+        for h in range(g.Hd):
+            for i in range(g.nb):
+                win = set()
+                if wl >= 0 or wr >= 0:
+                    lo = 0 if wl < 0 else i - wl
+                    hi = g.nb - 1 if wr < 0 else i + wr
+                    win = set(range(max(lo, 0), min(hi, g.nb - 1) + 1))
+                out[(b, h, i)] = win | sink | intra_sets[b][h]
+    return out
+
+
+def check_union_lists(g, gpu_idx, gpu_cnt, o_idx, o_cnt, tie, p, mode, params, extras,
+                      loose_heads=()):
+    """Lists of the mask union: bit-exact on non-tie rows.  On rows the oracle
+    flags as inter ties, the list must be E plus a valid inter selection S
+    (tie tolerance as check_lists).  Heads in loose_heads (an intra near-tie
+    under the SICS error bound) must contain their window and sink blocks.
+    Returns the number of tie rows."""
+    gi, gc = gpu_idx.cpu().numpy(), gpu_cnt.cpu().numpy()
+    n_tie = 0
+    text = list(range(g.nb, g.nb + g.nb_text))
+    for b in range(g.B):
+        for h in range(g.Hd):
+            for i in range(g.nb):
+                c = int(gc[b, h, i])
+                lst = [int(x) for x in gi[b, h, i, :c]]
+                ref = [int(x) for x in o_idx[b, h, i, :o_cnt[b, h, i]]]
+                if lst == ref:
+                    continue
+                assert lst[c - g.nb_text:] == text
+                L = lst[:c - g.nb_text]
+                assert all(x < y for x, y in zip(L, L[1:])) and (not L or (L[0] >= 0 and L[-1] < g.nb))
+                if (b, h) in loose_heads:
+                    continue
+                assert tie[b, h, i], f"union list mismatch at b={b} h={h} i={i}"
+                n_tie += 1
+                E = extras[(b, h, i)]
+                Ls = set(L)
+                assert E <= Ls
+                row = p[b, h, i]
+                must = sorted(Ls - E)
+                opt = sorted(Ls & E, key=lambda j: (-row[j], j))
+                if mode == 0:
+                    k = orc.k_for_density(params[h], g.nb)
+                    assert len(must) <= k
+                    S = set(must) | set(opt[:k - len(must)])
+                    assert len(S) == k
+                else:
+                    S = set(must)
+                    for j in opt:
+                        if S and row[sorted(S)].sum() >= params[h] * (1 - TIE_REL):
+                            break
+                        S.add(j)
+                    mass = row[list(S)].sum()
+                    assert mass >= params[h] * (1 - TIE_REL)
+                    assert mass - row[list(S)].min() < params[h] * (1 + TIE_REL)
+                uns = np.setdiff1d(np.arange(g.nb), np.array(sorted(S)))
+                if len(uns):
+                    assert row[sorted(S)].min() >= row[uns].max() * (1 - TIE_REL) - 1e-300
+    return n_tie
+
+
+def intra_near_tie(values, tol, mode, param):
+    """True when the Top-K / Top-P decision on `values` could change within
+    per-entry error bounds `tol` (both 1-D)."""
+    nb = len(values)
+    order = sorted(range(nb), key=lambda j: (-values[j], j))
+    v = np.asarray(values, dtype=np.float64)[order]
+    t = np.asarray(tol, dtype=np.float64)[order]
+    if mode == 0:
+        m = orc.k_for_density(param, nb)
+    else:
+        target = param * v.sum()
+        c = np.cumsum(v)
+        m = int(np.searchsorted(c, target, side="left")) + 1
+        m = min(max(m, 1), nb)
+        slack = param * t.sum() + t.sum()
+        if abs(c[m - 1] - target) <= slack or (m >= 2 and abs(c[m - 2] - target) <= slack):
+            return True
+    return m < nb and v[m - 1] - v[m] <= t[m - 1] + t[m]
