@@ -55,6 +55,8 @@ def _load():
         lib.orc_attention.argtypes = [P, P, P, P, P, P, ctypes.c_int, P, ctypes.c_longlong, P]
         lib.orc_select_union.argtypes = [P, P, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int, P,
                                          ctypes.c_int, ctypes.c_int, ctypes.c_longlong, P, P, P]
+        lib.orc_box_summaries.argtypes = [P, P, P]
+        lib.orc_scores_box.argtypes = [P, P, P, ctypes.c_int, P]
         lib.orc_sics.argtypes = [P, P, P]
         lib.orc_sics_online.argtypes = [P, P, P]
         lib.orc_aggregation_score.argtypes = [P, P, P]
@@ -123,6 +125,24 @@ def scores(g: Geometry, qc, kc):
     kc = np.ascontiguousarray(kc, dtype=np.float64)
     out = np.empty((g.B, g.Hd, g.nb, g.nb), dtype=np.float64)
     _load().orc_scores(_ptr(g.arr), _ptr(qc), _ptr(kc), _ptr(out))
+    return out
+
+
+def box_summaries(g: Geometry, x):
+    """Per video block and dimension (max, min) over valid tokens, [B,Hd,nb,D,2]
+    (SPADE §3.1 DSA / DSA2 summaries)."""
+    x = _f32(x)
+    out = np.empty((g.B, g.Hd, g.nb, g.D, 2), dtype=np.float64)
+    _load().orc_box_summaries(_ptr(g.arr), _ptr(x), _ptr(out))
+    return out
+
+
+def scores_box(g: Geometry, qbox, kbox, variant: int):
+    """Row softmax of the DSA (variant 1) or DSA2 (variant 2) estimate / sqrt(D)."""
+    qbox = np.ascontiguousarray(qbox, dtype=np.float64)
+    kbox = np.ascontiguousarray(kbox, dtype=np.float64)
+    out = np.empty((g.B, g.Hd, g.nb, g.nb), dtype=np.float64)
+    _load().orc_scores_box(_ptr(g.arr), _ptr(qbox), _ptr(kbox), int(variant), _ptr(out))
     return out
 
 
@@ -240,10 +260,13 @@ def selected_pairs(g: Geometry, idx, cnt) -> int:
     return int(_load().orc_selected_pairs(_ptr(g.arr), _ptr(idx), _ptr(cnt), idx.shape[-1]))
 
 
-def forward(g: Geometry, q, k, v, mode: int, params, rows=None):
-    """The whole executor: centroids -> scores -> selection -> attention."""
-    qc, kc = centroids(g, q), centroids(g, k)
-    p = scores(g, qc, kc)
+def forward(g: Geometry, q, k, v, mode: int, params, rows=None, estimator: int = 0):
+    """The whole executor: summaries -> scores -> selection -> attention
+    (estimator 0 = MEAN, 1 = DSA, 2 = DSA2)."""
+    if estimator == 0:
+        p = scores(g, centroids(g, q), centroids(g, k))
+    else:
+        p = scores_box(g, box_summaries(g, q), box_summaries(g, k), estimator)
     idx, cnt, tie = select(g, p, mode, params)
     o = attention(g, q, k, v, idx, cnt, rows=rows)
     return o, idx, cnt, tie, p

@@ -43,6 +43,8 @@
 //       the original sequence.
 //   R20 intra scores: one per key block, broadcast to every query block of
 //       the head; selected by the Top-K / Top-P rule on the scores.
+//   R21 DSA / DSA2 inter-estimators: the largest q . k over the summaries'
+//       boxes (DSA: query fixed at the box centre).
 //
 // Geometry array g[10] = {B, T, H, W, bf, br, bc, Hd, D, n_text}.
 
@@ -428,6 +430,71 @@ void orc_attention(const int* g, const float* q, const float* k, const float* v,
       double w = s[c] / z;
       for (long long d = 0; d < G.D; ++d) out[d] += w * (double)vv[d];
     }
+  });
+}
+
+// Box summarizer (SPADE §3.1 DSA-SPADE / DSA2-SPADE summaries k_max, k_min,
+// q_max, q_min; §3.2 "The Summarizer Expression reduces over sequence
+// positions of Q/K (e.g., max/min/mean)"): per video block and dimension the
+// maximum and the minimum over the block's valid tokens.
+// x [B, Ntot, Hd, D] -> box [B, Hd, nb, D, 2] with (max, min) pairs.
+void orc_box_summaries(const int* g, const float* x, double* box) {
+  Geom G = make_geom(g);
+  parallel_for(G.B * G.Hd * G.nb, [&](long long task) {
+    long long b = task / (G.Hd * G.nb), h = (task / G.nb) % G.Hd, j = task % G.nb;
+    std::vector<long long> toks = block_tokens(G, j);
+    double* out = box + task * G.D * 2;
+    for (long long d = 0; d < G.D; ++d) {
+      double mx = -INFINITY, mn = INFINITY;
+      for (long long t : toks) {
+        double v = (double)x[((b * G.n_tot + t) * G.Hd + h) * G.D + d];
+        mx = std::max(mx, v);
+        mn = std::min(mn, v);
+      }
+      out[2 * d] = mx;
+      out[2 * d + 1] = mn;
+    }
+  });
+}
+
+// Inter-block scores from box summaries, then the row softmax (R4).
+// variant 1, DSA-SPADE (estimate with (k_max, k_min, (q_max + q_min)/2)),
+//   reading R21: the largest value of c . k over the key block's box,
+//   c = (q_max + q_min) / 2, i.e. sum_d max(c_d k_max_d, c_d k_min_d);
+// variant 2, DSA2-SPADE (estimate with (k_max, k_min, q_max, q_min)),
+//   reading R21: the largest value of q . k over the query box times the key
+//   box, i.e. sum_d max over the four corner products of dimension d;
+// s_ij = estimate / sqrt(D), p_i = softmax_j(s_i).
+void orc_scores_box(const int* g, const double* qbox, const double* kbox, int variant,
+                    double* p) {
+  Geom G = make_geom(g);
+  const double scale = 1.0 / std::sqrt((double)G.D);
+  parallel_for(G.B * G.Hd * G.nb, [&](long long row) {
+    long long bh = row / G.nb;
+    const double* qb = qbox + row * G.D * 2;
+    double* pr = p + row * G.nb;
+    for (long long j = 0; j < G.nb; ++j) {
+      const double* kb = kbox + (bh * G.nb + j) * G.D * 2;
+      double est = 0.0;
+      for (long long d = 0; d < G.D; ++d) {
+        const double qM = qb[2 * d], qm = qb[2 * d + 1], kM = kb[2 * d], km = kb[2 * d + 1];
+        if (variant == 1) {
+          const double c = (qM + qm) / 2.0;
+          est += std::max(c * kM, c * km);
+        } else {
+          est += std::max(std::max(qM * kM, qM * km), std::max(qm * kM, qm * km));
+        }
+      }
+      pr[j] = est * scale;
+    }
+    double mx = -INFINITY;
+    for (long long j = 0; j < G.nb; ++j) mx = std::max(mx, pr[j]);
+    double z = 0.0;
+    for (long long j = 0; j < G.nb; ++j) {
+      pr[j] = std::exp(pr[j] - mx);
+      z += pr[j];
+    }
+    for (long long j = 0; j < G.nb; ++j) pr[j] /= z;
   });
 }
 

@@ -438,3 +438,77 @@ def test_union_intra_ties_are_flagged():
     v[0, 0, 5] = v[0, 0, 6]                        # k = 2 cut between two equal scores
     _, _, tie = orc.select_union(g, p, 0, [0.25, 0.25], intra=v, intra_params=[0.25, 0.25])
     assert tie[0, 0].all()
+
+
+# ---------------------------------------- DSA / DSA2 pins (SPADE §3.1, Fig. 4)
+@pytest.mark.parametrize("geo", [EVEN, RAGGED])
+def test_box_summaries_are_max_and_min_over_valid_tokens(geo):
+    g = orc.Geometry(**geo)
+    x = rand_x(g, 30)
+    Tp, Hp, Wp = g.nbt * g.bf, g.nby * g.br, g.nbx * g.bc
+    grid = np.full((g.B, Tp, Hp, Wp, g.Hd, g.D), np.nan)
+    grid[:, :g.T, :g.H, :g.W] = x[:, :g.n_video].reshape(g.B, g.T, g.H, g.W, g.Hd, g.D)
+    blk = grid.reshape(g.B, g.nbt, g.bf, g.nby, g.br, g.nbx, g.bc, g.Hd, g.D)
+    mx = np.nanmax(blk, axis=(2, 4, 6)).reshape(g.B, g.nb, g.Hd, g.D).transpose(0, 2, 1, 3)
+    mn = np.nanmin(blk, axis=(2, 4, 6)).reshape(g.B, g.nb, g.Hd, g.D).transpose(0, 2, 1, 3)
+    box = orc.box_summaries(g, x)
+    assert np.array_equal(box[..., 0], mx) and np.array_equal(box[..., 1], mn)
+
+
+def _corners(lo, hi):
+    """All 2^D corners of the box [lo, hi]."""
+    D = len(lo)
+    for bits in itertools.product((0, 1), repeat=D):
+        yield np.where(np.array(bits) == 1, hi, lo)
+
+
+def test_dsa_estimate_is_max_over_key_box_corners():
+    g = orc.Geometry(B=1, T=2, H=4, W=4, bf=1, br=2, bc=4, Hd=2, D=6, n_text=0)
+    x_q, x_k = rand_x(g, 31), rand_x(g, 32)
+    qb, kb = orc.box_summaries(g, x_q), orc.box_summaries(g, x_k)
+    p = orc.scores_box(g, qb, kb, 1)
+    for h in range(g.Hd):
+        for i in range(g.nb):
+            c = (qb[0, h, i, :, 0] + qb[0, h, i, :, 1]) / 2
+            est = np.array([max(c @ k for k in _corners(kb[0, h, j, :, 1], kb[0, h, j, :, 0]))
+                            for j in range(g.nb)]) / math.sqrt(g.D)
+            np.testing.assert_allclose(p[0, h, i], scipy.special.softmax(est), rtol=1e-12)
+
+
+def test_dsa2_estimate_is_max_over_both_boxes():
+    g = orc.Geometry(B=1, T=2, H=2, W=4, bf=1, br=2, bc=2, Hd=1, D=4, n_text=0)
+    x_q, x_k = rand_x(g, 33), rand_x(g, 34)
+    qb, kb = orc.box_summaries(g, x_q), orc.box_summaries(g, x_k)
+    p = orc.scores_box(g, qb, kb, 2)
+    for i in range(g.nb):
+        qs = list(_corners(qb[0, 0, i, :, 1], qb[0, 0, i, :, 0]))
+        est = np.array([max(qv @ kv for qv in qs for kv in _corners(kb[0, 0, j, :, 1], kb[0, 0, j, :, 0]))
+                        for j in range(g.nb)]) / math.sqrt(g.D)
+        np.testing.assert_allclose(p[0, 0, i], scipy.special.softmax(est), rtol=1e-12)
+
+
+def test_box_estimates_bound_the_token_dot_products():
+    # DSA2 >= every q_a . k_b of the two blocks; DSA >= every c . k_b
+    g = orc.Geometry(**dict(RAGGED, B=1, n_text=0))
+    x_q, x_k = rand_x(g, 35), rand_x(g, 36)
+    qb, kb = orc.box_summaries(g, x_q), orc.box_summaries(g, x_k)
+    tab = token_table(g)
+    for h in range(g.Hd):
+        for i in range(g.nb):
+            qa = x_q[0, tab[i][tab[i] >= 0], h].astype(np.float64)
+            c = (qb[0, h, i, :, 0] + qb[0, h, i, :, 1]) / 2
+            for j in range(g.nb):
+                kk = x_k[0, tab[j][tab[j] >= 0], h].astype(np.float64)
+                e1 = np.maximum(c * kb[0, h, j, :, 0], c * kb[0, h, j, :, 1]).sum()
+                q4 = np.stack([qb[0, h, i, :, 0] * kb[0, h, j, :, 0], qb[0, h, i, :, 0] * kb[0, h, j, :, 1],
+                               qb[0, h, i, :, 1] * kb[0, h, j, :, 0], qb[0, h, i, :, 1] * kb[0, h, j, :, 1]])
+                e2 = q4.max(0).sum()
+                assert e1 >= (kk @ c).max() - 1e-9
+                assert e2 >= (qa @ kk.T).max() - 1e-9
+    # one-token blocks: the boxes are points, both estimates are the dot product
+    g1 = orc.Geometry(B=1, T=1, H=2, W=3, bf=1, br=1, bc=1, Hd=1, D=5, n_text=0)
+    xq, xk = rand_x(g1, 37), rand_x(g1, 38)
+    dots = xq[0, :, 0].astype(np.float64) @ xk[0, :, 0].astype(np.float64).T / math.sqrt(5)
+    for v in (1, 2):
+        p = orc.scores_box(g1, orc.box_summaries(g1, xq), orc.box_summaries(g1, xk), v)
+        np.testing.assert_allclose(p[0, 0], scipy.special.softmax(dots, axis=-1), rtol=1e-12)
