@@ -238,6 +238,51 @@ def time_union_forward(bsa, w, plan, qd, kd, vd, out, dev, args, barrier):
             "mean_list_len": round(float(cnt.float().mean()), 2), "selected_pairs": pairs}
 
 
+def time_estimators(bsa, w, plan, qd, kd, vd, out, dev, args, barrier):
+    """Per box estimator (DSA, DSA2): CUDA-event times of the whole
+    bsa_forward_estimator step and of its summarizer and selection phases."""
+    L = bsa.load()
+    P = bsa._ptr
+    params = bsa._params(w.params, w.Hd)
+    kmax = plan.kmax_for(w.mode, w.params)
+    idx = torch.empty((w.B, w.Hd, plan.info.nb, kmax), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.B, w.Hd, plan.info.nb), dtype=torch.int32, device=dev)
+    qb, kb = (torch.empty(plan.box_shape, dtype=torch.float32, device=dev) for _ in range(2))
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    for name, est in (("dsa", 1), ("dsa2", 2)):
+        z = ctypes.c_size_t()
+        bsa._check(L.bsa_estimator_workspace_size(plan._h, est, kmax, None, ctypes.byref(z)))
+        ws = torch.empty(z.value, dtype=torch.uint8, device=dev)
+        calls = [
+            lambda: L.bsa_box_summaries(plan._h, P(qd), P(kd), P(qb), P(kb), bsa._stream(dev)),
+            lambda: L.bsa_select_box(plan._h, est, P(qb), P(kb), w.mode, params, None, None, kmax,
+                                     P(idx), P(cnt), None, None, 0, bsa._stream(dev)),
+            lambda: L.bsa_forward_estimator(plan._h, P(qd), P(kd), P(vd), est, w.mode, params, None,
+                                            kmax, P(out), P(idx), P(cnt), P(ws), ws.numel(), None,
+                                            bsa._stream(dev)),
+        ]
+        times = []
+        for c in calls:
+            for _ in range(args.warmup):
+                bsa._check(c())
+            barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                bsa._check(c())
+            e1.record(stream)
+            barrier()
+            times.append(e0.elapsed_time(e1) / args.steps)
+        plan.check_status()
+        pairs = effective_pairs(plan, idx, cnt)
+        res[name] = {"summaries_ms": round(times[0], 4), "select_ms": round(times[1], 4),
+                     "ms_per_step": round(times[2], 4),
+                     "tflops": round(4.0 * pairs * w.D / (times[2] * 1e-3) / 1e12, 2)}
+        del ws
+    return res
+
+
 CANDIDATE_SHAPES = [(1, 8, 16), (4, 4, 8), (16, 1, 8), (2, 8, 8), (8, 2, 8)]
 
 
@@ -389,6 +434,9 @@ def run_ours(args, rank, world, local):
     del qb, kb, vb, ob
     phase_ms = fused if fused is not None else unfused
 
+    # ---- the DSA / DSA2 box estimators in place of MEAN
+    estimators = time_estimators(bsa, w, plan, qd, kd, vd, out, dev, args, barrier)
+
     # ---- forward with the mask union (window, sink, intra blocks added)
     union = time_union_forward(bsa, w, plan, qd, kd, vd, out, dev, args, barrier)
 
@@ -526,6 +574,7 @@ def run_ours(args, rank, world, local):
                 "serial": {"value": round(job_tflops(world, flops, e2e_serial_ms), 2),
                            "ms_per_step": round(e2e_serial_ms, 3)}},
         "mask_union": dict(union, frac_of_peak=round(union["tflops"] / peak_tf, 4)),
+        "estimators": estimators,
         "scheme_generation": dict(scheme, share_of_attn=round(scheme["ms"] / phase_ms["attention"], 4),
                                   frac=round(scheme["achieved_gbs"] / hbm_gbs, 4),
                                   peak_gbs=hbm_gbs, bound="hbm"),

@@ -81,6 +81,10 @@ def load():
         "bsa_union_workspace_size": [P, I, P, ctypes.POINTER(Z), ctypes.POINTER(Z)],
         "bsa_select_union": [P, P, P, I, P, P, P, I, P, P, P, P, Z, P],
         "bsa_forward_union": [P, P, P, P, I, P, P, I, P, P, P, P, Z, P, P],
+        "bsa_box_summaries": [P, P, P, P, P, P],
+        "bsa_select_box": [P, I, P, P, I, P, P, P, I, P, P, P, P, Z, P],
+        "bsa_estimator_workspace_size": [P, I, I, P, ctypes.POINTER(Z)],
+        "bsa_forward_estimator": [P, P, P, P, I, I, P, P, I, P, P, P, P, Z, P, P],
         "bsa_aggregation_scores": [P, I, P, P, P, P, P],
     }
     for name, args in sigs.items():
@@ -359,6 +363,57 @@ class Plan:
                                         ctypes.byref(union) if union is not None else None, kmax,
                                         _ptr(out), _ptr(idx), _ptr(cnt), _ptr(ws), ws.numel(),
                                         _ptr(dev_status), _stream(self.device)))
+        return out, idx, cnt
+
+    # ---------------------------------------------------- box estimators
+    @property
+    def box_shape(self):
+        i = self.info
+        return (i.batch, i.heads, i.nb, i.head_dim, 2)
+
+    def box_summaries(self, q, k):
+        """(max, min) per video block and dimension of Q and K (bsa_box_summaries)."""
+        self._check_tensor(q, self.orig_shape, name="q")
+        self._check_tensor(k, self.orig_shape, name="k")
+        qb, kb = (self._new(self.box_shape, torch.float32) for _ in range(2))
+        _check(load().bsa_box_summaries(self._h, _ptr(q), _ptr(k), _ptr(qb), _ptr(kb),
+                                        _stream(self.device)))
+        return qb, kb
+
+    def select_box(self, est, q_box, k_box, mode, params, union=None, intra_scores=None,
+                   kmax=None, scores=False):
+        """bsa_select_box: lists from the DSA (est 1) or DSA2 (est 2) estimator."""
+        i = self.info
+        self._check_tensor(q_box, self.box_shape, torch.float32, "q_box")
+        self._check_tensor(k_box, self.box_shape, torch.float32, "k_box")
+        kmax = kmax or self.kmax_for_union(mode, params, union)
+        idx, cnt = self._lists(kmax)
+        sc = self._new((i.batch, i.heads, i.nb, i.nb), torch.float32) if scores else None
+        sel_ws = self.union_workspace_size(kmax, union)[0] if union is not None else 0
+        ws = self._new((max(sel_ws, 1),), torch.uint8)
+        _check(load().bsa_select_box(self._h, est, _ptr(q_box), _ptr(k_box), mode,
+                                     _params(params, i.heads),
+                                     ctypes.byref(union) if union is not None else None,
+                                     _ptr(intra_scores), kmax, _ptr(idx), _ptr(cnt), _ptr(sc),
+                                     _ptr(ws), ws.numel(), _stream(self.device)))
+        return (idx, cnt, sc) if scores else (idx, cnt)
+
+    def forward_estimator(self, q, k, v, est, mode, params, union=None, kmax=None, out=None,
+                          dev_status=None):
+        """bsa_forward_estimator: the whole path with MEAN / DSA / DSA2; returns (o, idx, cnt)."""
+        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+            self._check_tensor(t, self.orig_shape, name=n)
+        kmax = kmax or self.kmax_for_union(mode, params, union)
+        idx, cnt = self._lists(kmax)
+        out = self._new(self.orig_shape) if out is None else out
+        z = ctypes.c_size_t()
+        u = ctypes.byref(union) if union is not None else None
+        _check(load().bsa_estimator_workspace_size(self._h, est, kmax, u, ctypes.byref(z)))
+        ws = self._new((max(z.value, 1),), torch.uint8)
+        _check(load().bsa_forward_estimator(self._h, _ptr(q), _ptr(k), _ptr(v), est, mode,
+                                            _params(params, self.info.heads), u, kmax, _ptr(out),
+                                            _ptr(idx), _ptr(cnt), _ptr(ws), ws.numel(),
+                                            _ptr(dev_status), _stream(self.device)))
         return out, idx, cnt
 
     def check_status(self):

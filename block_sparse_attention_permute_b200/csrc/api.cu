@@ -216,7 +216,7 @@ bsa_status check_union(const bsa_plan_s* p, const bsa_mask_union_t* u, UnionOpts
 bsa_status run_select(const bsa_plan_s* p, const float* qc, const float* kc, bsa_select_mode mode,
                       const double* param, int kmax, int32_t* idx, int32_t* cnt, float* scores,
                       cudaStream_t st, const UnionOpts* uo = nullptr, const float* intra_scores = nullptr,
-                      uint32_t* bits = nullptr) {
+                      uint32_t* bits = nullptr, int est = bsa::kEstMean) {
   int need = 0;
   bsa_status s = check_params(p, mode, param, &need);
   if (s != BSA_OK) return s;
@@ -224,11 +224,14 @@ bsa_status run_select(const bsa_plan_s* p, const float* qc, const float* kc, bsa
   if (kmax < need) return fail(BSA_ERR_INVALID_ARG, "kmax %d is below the %d entries a list can need", kmax, need);
   if (p->g.nb == 0) return BSA_OK;
   if (!qc || !kc || !idx || !cnt) return fail(BSA_ERR_INVALID_ARG, "NULL centroid or list pointer");
-  if (!aligned16(qc) || !aligned16(kc)) return fail(BSA_ERR_INVALID_ARG, "centroids must be 16-byte aligned");
+  if (!aligned16(qc) || !aligned16(kc)) return fail(BSA_ERR_INVALID_ARG, "summaries must be 16-byte aligned");
+  if (est != bsa::kEstMean && bsa::select_smem_bytes(p->g.nb, 2 * p->g.D) > 227 * 1024)
+    return fail(BSA_ERR_UNSUPPORTED, "nb = %d is too large for the box estimators", p->g.nb);
   bsa::SelectArgs a;
   std::memset(&a, 0, sizeof(a));
   a.qc = qc; a.kc = kc; a.idx = idx; a.cnt = cnt; a.scores = scores; a.kmax = kmax;
   a.mode = (int)mode;
+  a.est = est;
   a.scale = (float)(1.0 / std::sqrt((double)p->g.D));
   for (int h = 0; h < p->g.Hd; ++h)
     a.param[h] = mode == BSA_TOPK ? (double)k_for_density(param[h], p->g.nb) : param[h];
@@ -284,14 +287,22 @@ bsa_status run_attention(const bsa_plan_s* p, const void* q, const void* k, cons
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "attention kernel");
 }
 
+// Summaries straight from the original layout: centroids (MEAN) or (max,
+// min) boxes (DSA, DSA2) of Q and K, optionally with the SICS of the K blocks.
 bsa_status run_centroids(const bsa_plan_s* p, const void* q, const void* k, float* qc, float* kc,
-                         cudaStream_t st, float* k_sics = nullptr) {
+                         cudaStream_t st, float* k_sics = nullptr, bool boxes = false) {
   // Only the requested tensors are read.
   bsa::GatherArgs ga;
   std::memset(&ga, 0, sizeof(ga));
-  if (qc) { ga.src[ga.ntensors] = q; ga.cent[ga.ntensors] = qc; ++ga.ntensors; }
+  if (qc) {
+    ga.src[ga.ntensors] = q;
+    (boxes ? ga.box : ga.cent)[ga.ntensors] = qc;
+    ++ga.ntensors;
+  }
   if (kc) {
-    ga.src[ga.ntensors] = k; ga.cent[ga.ntensors] = kc; ga.sics[ga.ntensors] = k_sics;
+    ga.src[ga.ntensors] = k;
+    (boxes ? ga.box : ga.cent)[ga.ntensors] = kc;
+    ga.sics[ga.ntensors] = k_sics;
     ++ga.ntensors;
   }
   if (ga.ntensors == 0 || p->g.nb == 0) return BSA_OK;
@@ -346,10 +357,11 @@ bsa_status run_forward_fused(const bsa_plan_s* p, const void* q, const void* k, 
                              bsa_select_mode mode, const double* param, int kmax, void* o,
                              int32_t* idx, int32_t* cnt, float* qc, float* kc,
                              int32_t* dev_status, cudaStream_t st, const UnionOpts* uo = nullptr,
-                             float* k_sics = nullptr, uint32_t* bits = nullptr) {
-  bsa_status s = run_centroids(p, q, k, qc, kc, st, k_sics);
+                             float* k_sics = nullptr, uint32_t* bits = nullptr,
+                             int est = bsa::kEstMean) {
+  bsa_status s = run_centroids(p, q, k, qc, kc, st, k_sics, est != bsa::kEstMean);
   if (s != BSA_OK) return s;
-  if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st, uo, k_sics, bits)) != BSA_OK)
+  if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st, uo, k_sics, bits, est)) != BSA_OK)
     return s;
   return run_attention_orig(p, q, k, v, idx, cnt, kmax, o, dev_status, st);
 }
@@ -368,12 +380,27 @@ bsa_status union_kmax(const bsa_plan_s* p, bsa_select_mode mode, const double* p
   return BSA_OK;
 }
 
+// Workspace of the forward: bsa_forward's (blocked tensors on SIMT plans,
+// two summary arrays sized for centroids, the lists), plus two more
+// centroid-sized arrays for box summaries (twice as wide), plus the K-block
+// SICS and intra bit sets when the union has an intra part.
+size_t forward_ws_bytes(const bsa_plan_s* p, int kmax, int est, bool intra) {
+  size_t base = 0;
+  bsa_workspace_size(const_cast<bsa_plan_s*>(p), kmax, nullptr, &base);
+  if (est != bsa::kEstMean) base += 2 * round256(cent_bytes(p));
+  if (intra) base += round256(bits_bytes(p)) + round256(sics_bytes(p));
+  return base;
+}
+
 bsa_status forward_impl(bsa_plan_t p, const void* q, const void* k, const void* v,
                         bsa_select_mode mode, const double* param, const bsa_mask_union_t* u,
                         int kmax, void* o, int32_t* idx_out, int32_t* cnt_out, void* ws,
-                        size_t ws_bytes, int32_t* dev_status, void* stream) {
+                        size_t ws_bytes, int32_t* dev_status, void* stream,
+                        int est = bsa::kEstMean) {
   bsa_status s = check_plan(p);
   if (s != BSA_OK) return s;
+  if (est != bsa::kEstMean && est != bsa::kEstDsa && est != bsa::kEstDsa2)
+    return fail(BSA_ERR_INVALID_ARG, "bad estimator %d", est);
   int need = 0;
   if ((s = union_kmax(p, mode, param, u, &need)) != BSA_OK) return s;
   if (kmax < need) return fail(BSA_ERR_INVALID_ARG, "kmax %d is below the %d entries a list can need", kmax, need);
@@ -383,9 +410,7 @@ bsa_status forward_impl(bsa_plan_t p, const void* q, const void* k, const void* 
   if (!q || !k || !v || !o) return fail(BSA_ERR_INVALID_ARG, "NULL tensor pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
-  size_t base_ws = 0;
-  bsa_workspace_size(p, kmax, nullptr, &base_ws);
-  const size_t need_ws = base_ws + (uo.intra ? round256(bits_bytes(p)) + round256(sics_bytes(p)) : 0);
+  const size_t need_ws = forward_ws_bytes(p, kmax, est, uo.intra);
   if (ws == nullptr || ws_bytes < need_ws)
     return fail(BSA_ERR_WORKSPACE, "forward needs %zu bytes of workspace, got %zu", need_ws, ws_bytes);
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(BSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
@@ -401,6 +426,12 @@ bsa_status forward_impl(bsa_plan_t p, const void* q, const void* k, const void* 
   w += round256((size_t)p->g.B * p->g.Hd * p->g.nb * kmax * sizeof(int32_t));
   int32_t* cnt = reinterpret_cast<int32_t*>(w);
   w += round256((size_t)p->g.B * p->g.Hd * p->g.nb * sizeof(int32_t));
+  if (est != bsa::kEstMean) {
+    // box summaries are twice as wide as centroids: Q's box takes the two
+    // centroid slots, K's box the two extra slots
+    kc = reinterpret_cast<float*>(w);
+    w += 2 * cb;
+  }
   float* k_sics = nullptr;
   uint32_t* bits = nullptr;
   if (uo.intra) {
@@ -413,17 +444,21 @@ bsa_status forward_impl(bsa_plan_t p, const void* q, const void* k, const void* 
   const UnionOpts* up = u ? &uo : nullptr;
   if (p->attn_path == 1)
     return run_forward_fused(p, q, k, v, mode, param, kmax, o, idx, cnt, qc, kc, dev_status, st, up,
-                             k_sics, bits);
+                             k_sics, bits, est);
   bsa::GatherArgs a;
   std::memset(&a, 0, sizeof(a));
   a.src[0] = q; a.src[1] = k; a.src[2] = v;
   a.dst[0] = q_blk; a.dst[1] = k_blk; a.dst[2] = v_blk;
-  a.cent[0] = qc; a.cent[1] = kc;
+  if (est == bsa::kEstMean) {
+    a.cent[0] = qc; a.cent[1] = kc;
+  } else {
+    a.box[0] = qc; a.box[1] = kc;
+  }
   a.sics[1] = k_sics;
   a.ntensors = 3;
   cudaError_t e = bsa::launch_permute(p->g, p->dtype == BSA_BF16, a, st);
   if (e != cudaSuccess) return cuda_fail(e, "permute kernel");
-  if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st, up, k_sics, bits)) != BSA_OK)
+  if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st, up, k_sics, bits, est)) != BSA_OK)
     return s;
   if ((s = run_attention(p, q_blk, k_blk, v_blk, idx, cnt, kmax, o_blk, dev_status, st)) != BSA_OK) return s;
   return bsa_unpermute(p, o_blk, o, stream);
@@ -662,13 +697,69 @@ bsa_status bsa_union_workspace_size(bsa_plan_t p, int kmax, const bsa_mask_union
   int extra = 0;
   bsa_status s = check_union(p, u, &uo, &extra);
   if (s != BSA_OK) return s;
-  size_t base = 0;
-  if ((s = bsa_workspace_size(p, kmax, nullptr, &base)) != BSA_OK) return s;
-  const size_t add_sel = uo.intra ? round256(bits_bytes(p)) : 0;
-  const size_t add_fwd = uo.intra ? round256(bits_bytes(p)) + round256(sics_bytes(p)) : 0;
-  if (select_ws) *select_ws = add_sel;
-  if (forward_ws) *forward_ws = base + add_fwd;
+  if (select_ws) *select_ws = uo.intra ? round256(bits_bytes(p)) : 0;
+  if (forward_ws) *forward_ws = forward_ws_bytes(p, kmax, bsa::kEstMean, uo.intra);
   return BSA_OK;
+}
+
+bsa_status bsa_estimator_workspace_size(bsa_plan_t p, bsa_estimator est, int kmax,
+                                        const bsa_mask_union_t* u, size_t* forward_ws) {
+  if (p == nullptr) return fail(BSA_ERR_INVALID_ARG, "plan is NULL");
+  if (est != BSA_EST_MEAN && est != BSA_EST_DSA && est != BSA_EST_DSA2)
+    return fail(BSA_ERR_INVALID_ARG, "bad estimator %d", (int)est);
+  UnionOpts uo;
+  int extra = 0;
+  bsa_status s = check_union(p, u, &uo, &extra);
+  if (s != BSA_OK) return s;
+  if (forward_ws) *forward_ws = forward_ws_bytes(p, kmax, (int)est, uo.intra);
+  return BSA_OK;
+}
+
+bsa_status bsa_box_summaries(bsa_plan_t p, const void* q, const void* k, float* q_box,
+                             float* k_box, void* stream) {
+  bsa_status s = check_plan(p);
+  if (s != BSA_OK) return s;
+  if ((q_box && !q) || (k_box && !k)) return fail(BSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  const void* ptrs[4] = {q, k, q_box, k_box};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  return run_centroids(p, q, k, q_box, k_box, (cudaStream_t)stream, nullptr, true);
+}
+
+bsa_status bsa_select_box(bsa_plan_t p, bsa_estimator est, const float* q_box, const float* k_box,
+                          bsa_select_mode mode, const double* param, const bsa_mask_union_t* u,
+                          const float* intra_scores, int kmax, int32_t* idx, int32_t* cnt,
+                          float* scores, void* ws, size_t ws_bytes, void* stream) {
+  bsa_status s = check_plan(p);
+  if (s != BSA_OK) return s;
+  if (est != BSA_EST_DSA && est != BSA_EST_DSA2)
+    return fail(BSA_ERR_INVALID_ARG, "bsa_select_box needs BSA_EST_DSA or BSA_EST_DSA2");
+  int need = 0;
+  if ((s = union_kmax(p, mode, param, u, &need)) != BSA_OK) return s;
+  if (kmax < need) return fail(BSA_ERR_INVALID_ARG, "kmax %d is below the %d entries a list can need", kmax, need);
+  UnionOpts uo;
+  int extra = 0;
+  if ((s = check_union(p, u, &uo, &extra)) != BSA_OK) return s;
+  uint32_t* bits = nullptr;
+  if (uo.intra) {
+    if (intra_scores == nullptr) return fail(BSA_ERR_INVALID_ARG, "intra selection needs intra_scores");
+    if (ws == nullptr || ws_bytes < bits_bytes(p))
+      return fail(BSA_ERR_WORKSPACE, "union selection needs %zu bytes of workspace, got %zu",
+                  round256(bits_bytes(p)), ws_bytes);
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(BSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    bits = reinterpret_cast<uint32_t*>(ws);
+  }
+  return run_select(p, q_box, k_box, mode, param, kmax, idx, cnt, scores, (cudaStream_t)stream,
+                    u ? &uo : nullptr, intra_scores, bits, (int)est);
+}
+
+bsa_status bsa_forward_estimator(bsa_plan_t p, const void* q, const void* k, const void* v,
+                                 bsa_estimator est, bsa_select_mode mode, const double* param,
+                                 const bsa_mask_union_t* u, int kmax, void* o, int32_t* idx_out,
+                                 int32_t* cnt_out, void* ws, size_t ws_bytes, int32_t* dev_status,
+                                 void* stream) {
+  return forward_impl(p, q, k, v, mode, param, u, kmax, o, idx_out, cnt_out, ws, ws_bytes,
+                      dev_status, stream, (int)est);
 }
 
 bsa_status bsa_select_union(bsa_plan_t p, const float* q_cent, const float* k_cent,

@@ -10,6 +10,7 @@ struct GatherArgs {
   void* dst[3];      // unused in kPool
   float* cent[3];    // optional centroid outputs (kPermute, kPool)
   float* sics[3];    // optional SICS outputs [B, Hd, nb] (kPermute, kPool, kPoolOrig)
+  float* box[3];     // optional box summaries [B, Hd, nb, D, 2] = (max, min) (same modes)
   int ntensors;
 };
 
@@ -26,14 +27,20 @@ struct SchemeArgs {
   int n;
 };
 
+// Inter-estimators of the selection: MEAN dots the centroids; DSA dots
+// (c+, c-) of the query box centre c with the key box (max, min); DSA2 sums,
+// per dimension, the largest corner product of the two boxes.
+enum Estimator { kEstMean = 0, kEstDsa = 1, kEstDsa2 = 2 };
+
 struct SelectArgs {
-  const float* qc;   // [B, Hd, nb, D]
-  const float* kc;   // [B, Hd, nb, D]
+  const float* qc;   // [B, Hd, nb, D] centroids, or [B, Hd, nb, D, 2] boxes
+  const float* kc;   // same layout as qc
   int32_t* idx;      // [B, Hd, nb, kmax]
   int32_t* cnt;      // [B, Hd, nb]
   float* scores;     // [B, Hd, nb, nb] or null
   int kmax;
   int mode;          // 0 top-k, 1 top-p
+  int est;           // Estimator
   float scale;       // 1/sqrt(D) rounded to fp32
   double param[BSA_MAX_HEADS];  // k (held in a double) or tau, per head
   // Mask union (video key blocks added to every list of a head):

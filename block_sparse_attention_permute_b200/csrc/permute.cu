@@ -69,7 +69,8 @@ __device__ __forceinline__ void to_float(const uint4& v, float* f) {
 // non-negative.
 template <typename T, int D, int MODE>
 __device__ __forceinline__ void gather_block(const Geo& g, const void* src_ptr, void* dst_ptr,
-                                             float* cent_ptr, float* sics_ptr, int j, int h, int b) {
+                                             float* cent_ptr, float* sics_ptr, float* box_ptr,
+                                             int j, int h, int b) {
   constexpr int E = 16 / (int)sizeof(T);  // elements per 16-byte vector
   constexpr int V = D / E;                // vectors per row
   constexpr int R = kGatherThreads / V;   // rows per pass
@@ -86,9 +87,14 @@ __device__ __forceinline__ void gather_block(const Geo& g, const void* src_ptr, 
   const long long tok_base = (long long)b * g.n_tot;
   float* cent = (MODE != kUnpermute && j < g.nb) ? cent_ptr : nullptr;
   float* sics = (MODE != kUnpermute && j < g.nb) ? sics_ptr : nullptr;
-  float acc[E], racc[E];
+  float* box = (MODE != kUnpermute && j < g.nb) ? box_ptr : nullptr;
+  float acc[E], racc[E], vmax[E], vmin[E];
 #pragma unroll
-  for (int e = 0; e < E; ++e) acc[e] = racc[e] = 0.f;
+  for (int e = 0; e < E; ++e) {
+    acc[e] = racc[e] = 0.f;
+    vmax[e] = -INFINITY;
+    vmin[e] = INFINITY;
+  }
 
   const uint4* src = reinterpret_cast<const uint4*>(src_ptr);
   uint4* dst = reinterpret_cast<uint4*>(dst_ptr);
@@ -113,6 +119,15 @@ __device__ __forceinline__ void gather_block(const Geo& g, const void* src_ptr, 
       if (MODE == kPermute && tok[u] >= -1) dst[(blk_row0 + s) * V + vec] = buf[u];
       if (MODE == kUnpermute && tok[u] >= 0) dst[((tok_base + tok[u]) * g.Hd + h) * V + vec] = buf[u];
       if (MODE != kUnpermute && cent != nullptr && tok[u] >= 0) accumulate_vec<T>(acc, buf[u]);
+      if (MODE != kUnpermute && box != nullptr && tok[u] >= 0) {
+        float f[E];
+        to_float<T>(buf[u], f);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          vmax[e] = fmaxf(vmax[e], f[e]);
+          vmin[e] = fminf(vmin[e], f[e]);
+        }
+      }
       if (MODE != kUnpermute && sics != nullptr) {
         // Every lane takes part (pad and out-of-range rows hold zeros): the V
         // lanes of one row are an aligned group of the warp.
@@ -138,6 +153,24 @@ __device__ __forceinline__ void gather_block(const Geo& g, const void* src_ptr, 
       for (int r = 0; r < R; ++r) sum += s_red[r * D + tid];
       const float n = (float)block_valid_count(g, j);
       cent[((long long)(b * g.Hd + h) * g.nb + j) * D + tid] = sum / n;
+    }
+  }
+
+  if (MODE != kUnpermute && box != nullptr) {
+    // per dimension: max, then min, over the R row groups (exact in fp32)
+    float* out = box + ((long long)(b * g.Hd + h) * g.nb + j) * D * 2;
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+      __syncthreads();  // s_red is reused
+#pragma unroll
+      for (int e = 0; e < E; ++e) s_red[row0 * D + vec * E + e] = pass == 0 ? vmax[e] : vmin[e];
+      __syncthreads();
+      if (tid < D) {
+        float r = s_red[tid];
+        for (int rr = 1; rr < R; ++rr)
+          r = pass == 0 ? fmaxf(r, s_red[rr * D + tid]) : fminf(r, s_red[rr * D + tid]);
+        out[2 * tid + pass] = r;
+      }
     }
   }
 
@@ -173,7 +206,9 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(Geo g, GatherArg
   void* dst = t == 0 ? a.dst[0] : t == 1 ? a.dst[1] : a.dst[2];
   float* cent = t == 0 ? a.cent[0] : t == 1 ? a.cent[1] : a.cent[2];
   float* sics = t == 0 ? a.sics[0] : t == 1 ? a.sics[1] : a.sics[2];
-  gather_block<T, D, MODE>(g, src, dst, cent, sics, blockIdx.x, blockIdx.y, blockIdx.z / a.ntensors);
+  float* box = t == 0 ? a.box[0] : t == 1 ? a.box[1] : a.box[2];
+  gather_block<T, D, MODE>(g, src, dst, cent, sics, box, blockIdx.x, blockIdx.y,
+                           blockIdx.z / a.ntensors);
 }
 
 // Aggregation evaluation (SPADE §3.2): SICS of every block of every candidate

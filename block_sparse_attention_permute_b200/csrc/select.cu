@@ -167,7 +167,14 @@ __device__ __forceinline__ long long block_first_token(const Geo& g, int j) {
   return ((long long)tb * g.bf * g.H + (long long)yb * g.br) * g.W + (long long)xb * g.bc;
 }
 
-template <int D>
+// Largest product of a in [am, aM] and b in [bm, bM] (a corner of the box).
+__device__ __forceinline__ float box_max_product(float aM, float am, float bM, float bm) {
+  return fmaxf(fmaxf(aM * bM, aM * bm), fmaxf(am * bM, am * bm));
+}
+
+// D = length of the stored summary vectors (head_dim for MEAN, 2 * head_dim
+// for the (max, min) boxes of DSA and DSA2).
+template <int D, int EST>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, SelectArgs a) {
   extern __shared__ __align__(16) float sm[];
   float* qs = sm;                                   // [kSelRows][D]
@@ -184,9 +191,26 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, SelectArgs a
   // each 256-key chunk; the chunk's keys pass through shared memory 32
   // dimensions at a time.  Each dot product is one fma chain over d in
   // ascending order, the same as a plain sequential loop.
-  for (int e = tid; e < kSelRows * D; e += kSelThreads) {
-    const int r = e / D, d = e % D;
-    qs[e] = (i0 + r < nb) ? a.qc[(bh * nb + i0 + r) * D + d] : 0.f;
+  if (EST == kEstDsa) {
+    // DSA: the query summary is the box centre c = (max + min) / 2, stored as
+    // (c+, c-) pairs so that c+ kmax + c- kmin = max(c kmax, c kmin)
+    for (int e = tid; e < kSelRows * D / 2; e += kSelThreads) {
+      const int r = e / (D / 2), d = e % (D / 2);
+      float cp = 0.f, cn = 0.f;
+      if (i0 + r < nb) {
+        const float* src = a.qc + (bh * nb + i0 + r) * D + 2 * d;
+        const float c = 0.5f * (src[0] + src[1]);
+        cp = fmaxf(c, 0.f);
+        cn = fminf(c, 0.f);
+      }
+      qs[r * D + 2 * d] = cp;
+      qs[r * D + 2 * d + 1] = cn;
+    }
+  } else {
+    for (int e = tid; e < kSelRows * D; e += kSelThreads) {
+      const int r = e / D, d = e % D;
+      qs[e] = (i0 + r < nb) ? a.qc[(bh * nb + i0 + r) * D + d] : 0.f;
+    }
   }
   const int ty = tid / 128, tx = tid % 128;
   constexpr int KS = kSelDChunk + 4;               // padded row: conflict-free float4 reads
@@ -211,6 +235,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, SelectArgs a
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
           const float4 qv = *reinterpret_cast<const float4*>(qs + (8 * ty + r) * D + d0 + 4 * d4);
+          if (EST == kEstDsa2) {
+            acc[r][0] += box_max_product(qv.x, qv.y, k0.x, k0.y);
+            acc[r][0] += box_max_product(qv.z, qv.w, k0.z, k0.w);
+            acc[r][1] += box_max_product(qv.x, qv.y, k1.x, k1.y);
+            acc[r][1] += box_max_product(qv.z, qv.w, k1.z, k1.w);
+            continue;
+          }
           acc[r][0] = fmaf(qv.x, k0.x, acc[r][0]);
           acc[r][0] = fmaf(qv.y, k0.y, acc[r][0]);
           acc[r][0] = fmaf(qv.z, k0.z, acc[r][0]);
@@ -327,22 +358,27 @@ cudaError_t launch_intra_select(const Geo& g, const IntraArgs& a, cudaStream_t s
   return cudaGetLastError();
 }
 
-cudaError_t launch_select(const Geo& g, const SelectArgs& a, cudaStream_t st) {
-  const size_t smem = select_smem_bytes(g.nb, g.D);
+template <int D, int EST>
+static cudaError_t launch_select_t(const Geo& g, const SelectArgs& a, cudaStream_t st) {
+  const size_t smem = select_smem_bytes(g.nb, D);
   dim3 grid((g.nb + kSelRows - 1) / kSelRows, g.Hd, g.B);
-  cudaError_t e;
-  if (g.D == 128) {
-    e = cudaFuncSetAttribute(select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
-    select_kernel<128><<<grid, kSelThreads, smem, st>>>(g, a);
-  } else {
-    e = cudaFuncSetAttribute(select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
-    select_kernel<64><<<grid, kSelThreads, smem, st>>>(g, a);
-  }
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<D, EST>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  select_kernel<D, EST><<<grid, kSelThreads, smem, st>>>(g, a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_select(const Geo& g, const SelectArgs& a, cudaStream_t st) {
+  const bool d128 = g.D == 128;
+  switch (a.est) {
+    case kEstDsa:
+      return d128 ? launch_select_t<256, kEstDsa>(g, a, st) : launch_select_t<128, kEstDsa>(g, a, st);
+    case kEstDsa2:
+      return d128 ? launch_select_t<256, kEstDsa2>(g, a, st) : launch_select_t<128, kEstDsa2>(g, a, st);
+    default:
+      return d128 ? launch_select_t<128, kEstMean>(g, a, st) : launch_select_t<64, kEstMean>(g, a, st);
+  }
 }
 
 }  // namespace bsa

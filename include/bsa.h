@@ -354,6 +354,57 @@ bsa_status bsa_forward_union(bsa_plan_t plan, const void* q, const void* k,
                              size_t ws_bytes, int32_t* dev_status,
                              void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Inter-estimators (SPADE §3.1: DSA-SPADE estimates with
+ * (k_max, k_min, (q_max + q_min)/2), DSA2-SPADE with (k_max, k_min, q_max,
+ * q_min), MEAN-SPADE with (q_mean, k_mean); the estimator equations sit in
+ * the paper's Fig. 4, which its text does not reproduce).  Reading taken
+ * here: the box estimators bound the largest dot product a block pair can
+ * reach given the per-dimension (max, min) summaries of its blocks:
+ *   DSA   est_ij = sum_d max(c_d kmax_d, c_d kmin_d),  c = (qmax + qmin) / 2
+ *         (the largest c . k over the key block's box);
+ *   DSA2  est_ij = sum_d max(qmax_d kmax_d, qmax_d kmin_d, qmin_d kmax_d,
+ *         qmin_d kmin_d)  (the largest q . k over both boxes);
+ * s_ij = est_ij / sqrt(D), selected by Top-K / Top-P on softmax_j(s_i) as
+ * for MEAN.  The (max, min) are taken over the block's valid tokens. */
+typedef enum { BSA_EST_MEAN = 0, BSA_EST_DSA = 1, BSA_EST_DSA2 = 2 } bsa_estimator;
+
+/* bsa_box_summaries — per video block and dimension the (max, min) of the
+ * valid tokens, straight from the original layout.
+ *   q, k          [B, Ntot, Hd, D] original order (read only)
+ *   q_box, k_box  [B, Hd, nb, D, 2] float out, (max, min) pairs (either may
+ *                 be NULL) */
+bsa_status bsa_box_summaries(bsa_plan_t plan, const void* q, const void* k,
+                             float* q_box, float* k_box, void* stream);
+
+/* bsa_select_box — bsa_select_union with the DSA or DSA2 estimator on box
+ * summaries (as written by bsa_box_summaries).  est must be BSA_EST_DSA or
+ * BSA_EST_DSA2; u may be NULL; other arguments as bsa_select_union. */
+bsa_status bsa_select_box(bsa_plan_t plan, bsa_estimator est,
+                          const float* q_box, const float* k_box,
+                          bsa_select_mode mode, const double* param_per_head,
+                          const bsa_mask_union_t* u, const float* intra_scores,
+                          int kmax, int32_t* idx, int32_t* cnt, float* scores,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* bsa_estimator_workspace_size — workspace of bsa_forward_estimator. */
+bsa_status bsa_estimator_workspace_size(bsa_plan_t plan, bsa_estimator est,
+                                        int kmax, const bsa_mask_union_t* u,
+                                        size_t* forward_ws);
+
+/* bsa_forward_estimator — bsa_forward_union with the chosen inter-estimator:
+ * the summarizer pass writes centroids (MEAN) or boxes (DSA, DSA2), plus the
+ * K-block SICS when u has an intra part.  est = BSA_EST_MEAN is
+ * bsa_forward_union.  ws_bytes >= bsa_estimator_workspace_size. */
+bsa_status bsa_forward_estimator(bsa_plan_t plan, const void* q, const void* k,
+                                 const void* v, bsa_estimator est,
+                                 bsa_select_mode mode,
+                                 const double* param_per_head,
+                                 const bsa_mask_union_t* u, int kmax, void* o,
+                                 int32_t* idx_out, int32_t* cnt_out, void* ws,
+                                 size_t ws_bytes, int32_t* dev_status,
+                                 void* stream);
+
 /* bsa_check_status — synchronise `stream`, read and clear the plan-owned
  * status word; returns BSA_OK or the recorded error. */
 bsa_status bsa_check_status(bsa_plan_t plan, void* stream);

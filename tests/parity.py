@@ -29,8 +29,34 @@ def to_np(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy() if t.dtype == torch.bfloat16 else t.detach().cpu().numpy()
 
 
-def check_lists(g, gpu_idx, gpu_cnt, o_idx, o_cnt, tie, p, mode, params):
-    """Bit-exact lists on non-tie rows; valid selections on tie rows. Returns #ties."""
+def bound_ties(g, p, tol, mode, params):
+    """[B, Hd, nb] rows whose Top-K / Top-P cut could move when every p_ij may
+    be off by up to tol_ij (a derived error bound of the kernel's scores)."""
+    tie = np.zeros((g.B, g.Hd, g.nb), dtype=np.int32)
+    for b in range(g.B):
+        for h in range(g.Hd):
+            for i in range(g.nb):
+                row, t = p[b, h, i], tol[b, h, i]
+                order = np.lexsort((np.arange(g.nb), -row))
+                v, tv = row[order], t[order]
+                if mode == 0:
+                    m = orc.k_for_density(params[h], g.nb)
+                else:
+                    c = np.cumsum(v)
+                    m = min(int(np.searchsorted(c, params[h], side="left")) + 1, g.nb)
+                    slack = tv.sum()
+                    if abs(c[m - 1] - params[h]) <= slack or (m >= 2 and abs(c[m - 2] - params[h]) <= slack):
+                        tie[b, h, i] = 1
+                if m < g.nb and v[m - 1] - v[m] <= tv[m - 1] + tv[m]:
+                    tie[b, h, i] = 1
+    return tie
+
+
+def check_lists(g, gpu_idx, gpu_cnt, o_idx, o_cnt, tie, p, mode, params, tol=None):
+    """Bit-exact lists on non-tie rows; valid selections on tie rows. Returns #ties.
+
+    tol (optional, like p): per-score error bounds; tie rows must then be a
+    valid selection within those bounds instead of within TIE_REL."""
     gi, gc = gpu_idx.cpu().numpy(), gpu_cnt.cpu().numpy()
     assert gc.shape == o_cnt.shape
     n_tie = 0
@@ -50,15 +76,27 @@ def check_lists(g, gpu_idx, gpu_cnt, o_idx, o_cnt, tie, p, mode, params):
                 assert np.all(np.diff(sel) > 0) and sel.min() >= 0 and sel.max() < g.nb
                 row = p[b, h, i]
                 uns = np.setdiff1d(np.arange(g.nb), sel)
-                if len(uns):
-                    assert row[sel].min() >= row[uns].max() * (1 - TIE_REL) - 1e-300
-                if mode == 0:
-                    assert len(sel) == orc.k_for_density(params[h], g.nb)
+                if tol is None:
+                    if len(uns):
+                        assert row[sel].min() >= row[uns].max() * (1 - TIE_REL) - 1e-300
+                    if mode == 0:
+                        assert len(sel) == orc.k_for_density(params[h], g.nb)
+                    else:
+                        tau = params[h]
+                        mass = row[sel].sum()
+                        assert mass >= tau * (1 - TIE_REL)
+                        assert mass - row[sel].min() < tau * (1 + TIE_REL)
                 else:
-                    tau = params[h]
-                    mass = row[sel].sum()
-                    assert mass >= tau * (1 - TIE_REL)
-                    assert mass - row[sel].min() < tau * (1 + TIE_REL)
+                    t = tol[b, h, i]
+                    if len(uns):
+                        assert (row[sel] + t[sel]).min() >= (row[uns] - t[uns]).max()
+                    if mode == 0:
+                        assert len(sel) == orc.k_for_density(params[h], g.nb)
+                    else:
+                        tau, slack = params[h], t.sum()
+                        mass = row[sel].sum()
+                        assert mass >= tau - slack
+                        assert mass - row[sel].min() < tau + slack
     return n_tie
 
 
