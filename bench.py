@@ -283,6 +283,60 @@ def time_estimators(bsa, w, plan, qd, kd, vd, out, dev, args, barrier):
     return res
 
 
+def time_grouped_forward(bsa, w, qd, kd, vd, dev, args, barrier):
+    """Per-head blocking schemes: the aggregation-score choice among three
+    candidate block shapes (computed once), then CUDA-event timing of
+    bsa_forward_grouped over --steps steps."""
+    shapes = [(w.bf, w.br, w.bc)] + [s for s in CANDIDATE_SHAPES if s != (w.bf, w.br, w.bc)][:2]
+    plans = [bsa.Plan(w.B, w.T, w.H, w.W, a, b, c, w.Hd, w.D, w.n_text, qd.dtype, dev)
+             for a, b, c in shapes]
+    if any(p.info.attn_path != 1 for p in plans):
+        return {"skipped": "grouped forward needs tensor-core plans"}
+    _, _, choice = bsa.aggregation_scores(plans, qd)
+    head_plan = choice.cpu().flatten().tolist()
+    L = bsa.load()
+    n = len(plans)
+    kmaxes = [p.kmax_for(w.mode, w.params) for p in plans]
+    lists = [p._lists(km) for p, km in zip(plans, kmaxes)]
+    for _, cnt in lists:
+        cnt.zero_()
+    hp = (ctypes.c_int32 * len(head_plan))(*head_plan)
+    km = (ctypes.c_int * n)(*kmaxes)
+    hs = (ctypes.c_void_p * n)(*[p._h.value for p in plans])
+    ia = (ctypes.c_void_p * n)(*[l[0].data_ptr() for l in lists])
+    ca = (ctypes.c_void_p * n)(*[l[1].data_ptr() for l in lists])
+    z = ctypes.c_size_t()
+    bsa._check(L.bsa_grouped_workspace_size(hs, n, km, None, ctypes.byref(z)))
+    ws = torch.empty(z.value, dtype=torch.uint8, device=dev)
+    out = torch.empty_like(qd)
+    params = bsa._params(w.params, w.Hd)
+    P = bsa._ptr
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        bsa._check(L.bsa_forward_grouped(hs, n, hp, P(qd), P(kd), P(vd), w.mode, params, None, km,
+                                         P(out), ia, ca, P(ws), ws.numel(), None, bsa._stream(dev)))
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    plans[0].check_status()
+    i0 = plans[0].info
+    text = sum(min(i0.bs, i0.n_text - t * i0.bs) for t in range(i0.nb_text)) * i0.n_tot * w.B * w.Hd
+    pairs = text + sum(effective_pairs(p, idx, cnt) - text for p, (idx, cnt) in zip(plans, lists))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    return {"candidates": [f"{a}x{b}x{c}" for a, b, c in shapes],
+            "heads_per_scheme": [head_plan.count(c) for c in range(n)],
+            "ms_per_step": round(ms, 4), "effective_tflop_per_step": round(4.0 * pairs * w.D / 1e12, 4),
+            "tflops": round(4.0 * pairs * w.D / (ms * 1e-3) / 1e12, 2), "selected_pairs": pairs}
+
+
 CANDIDATE_SHAPES = [(1, 8, 16), (4, 4, 8), (16, 1, 8), (2, 8, 8), (8, 2, 8)]
 
 
@@ -440,6 +494,9 @@ def run_ours(args, rank, world, local):
     # ---- forward with the mask union (window, sink, intra blocks added)
     union = time_union_forward(bsa, w, plan, qd, kd, vd, out, dev, args, barrier)
 
+    # ---- per-head blocking schemes: grouped forward on the aggregation choice
+    grouped = time_grouped_forward(bsa, w, qd, kd, vd, dev, args, barrier)
+
     # ---- scheme generation (aggregation evaluation over candidate blockings):
     # one launch evaluates three candidate schemes of Q; timed alone.
     scheme = time_scheme_generation(bsa, w, qd, dev, args, barrier)
@@ -575,6 +632,7 @@ def run_ours(args, rank, world, local):
                            "ms_per_step": round(e2e_serial_ms, 3)}},
         "mask_union": dict(union, frac_of_peak=round(union["tflops"] / peak_tf, 4)),
         "estimators": estimators,
+        "scheme_adaptive": dict(grouped, frac_of_peak=round(grouped["tflops"] / peak_tf, 4)),
         "scheme_generation": dict(scheme, share_of_attn=round(scheme["ms"] / phase_ms["attention"], 4),
                                   frac=round(scheme["achieved_gbs"] / hbm_gbs, 4),
                                   peak_gbs=hbm_gbs, bound="hbm"),

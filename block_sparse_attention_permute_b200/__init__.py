@@ -85,6 +85,8 @@ def load():
         "bsa_select_box": [P, I, P, P, I, P, P, P, I, P, P, P, P, Z, P],
         "bsa_estimator_workspace_size": [P, I, I, P, ctypes.POINTER(Z)],
         "bsa_forward_estimator": [P, P, P, P, I, I, P, P, I, P, P, P, P, Z, P, P],
+        "bsa_grouped_workspace_size": [P, I, P, P, ctypes.POINTER(Z)],
+        "bsa_forward_grouped": [P, I, P, P, P, P, I, P, P, P, P, P, P, P, Z, P, P],
         "bsa_aggregation_scores": [P, I, P, P, P, P, P],
     }
     for name, args in sigs.items():
@@ -440,6 +442,40 @@ def aggregation_scores(plans, x):
     _check(load().bsa_aggregation_scores(handles, n, _ptr(x), outs, _ptr(as_), _ptr(choice),
                                          _stream(p0.device)))
     return sics, as_, choice
+
+
+def forward_grouped(plans, head_plan, q, k, v, mode, params, union=None, kmax=None, out=None):
+    """bsa_forward_grouped: each (b, h) served by plans[head_plan[b*Hd + h]].
+
+    head_plan: sequence or int tensor of B*Hd plan indices (host values).
+    Returns (o, lists) with lists[c] = (idx, cnt) of plan c (only its heads written).
+    """
+    plans = list(plans)
+    n = len(plans)
+    p0 = plans[0]
+    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+        p0._check_tensor(t, p0.orig_shape, name=nm)
+    hp = [int(x) for x in (head_plan.flatten().tolist() if isinstance(head_plan, torch.Tensor)
+                           else head_plan)]
+    hp_arr = (ctypes.c_int32 * len(hp))(*hp)
+    kmaxes = kmax or [p.kmax_for_union(mode, params, union) for p in plans]
+    km_arr = (ctypes.c_int * n)(*kmaxes)
+    lists = [p._lists(km) for p, km in zip(plans, kmaxes)]
+    for idx, cnt in lists:
+        cnt.zero_()
+    idx_arr = (ctypes.c_void_p * n)(*[l[0].data_ptr() for l in lists])
+    cnt_arr = (ctypes.c_void_p * n)(*[l[1].data_ptr() for l in lists])
+    handles = (ctypes.c_void_p * n)(*[p._h.value for p in plans])
+    u = ctypes.byref(union) if union is not None else None
+    z = ctypes.c_size_t()
+    _check(load().bsa_grouped_workspace_size(handles, n, km_arr, u, ctypes.byref(z)))
+    ws = p0._new((max(z.value, 1),), torch.uint8)
+    out = p0._new(p0.orig_shape) if out is None else out
+    _check(load().bsa_forward_grouped(handles, n, hp_arr, _ptr(q), _ptr(k), _ptr(v), mode,
+                                      _params(params, p0.info.heads), u, km_arr, _ptr(out),
+                                      idx_arr, cnt_arr, _ptr(ws), ws.numel(), None,
+                                      _stream(p0.device)))
+    return out, lists
 
 
 def plan_for(w, device=None) -> Plan:

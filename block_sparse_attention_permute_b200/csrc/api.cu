@@ -216,7 +216,8 @@ bsa_status check_union(const bsa_plan_s* p, const bsa_mask_union_t* u, UnionOpts
 bsa_status run_select(const bsa_plan_s* p, const float* qc, const float* kc, bsa_select_mode mode,
                       const double* param, int kmax, int32_t* idx, int32_t* cnt, float* scores,
                       cudaStream_t st, const UnionOpts* uo = nullptr, const float* intra_scores = nullptr,
-                      uint32_t* bits = nullptr, int est = bsa::kEstMean) {
+                      uint32_t* bits = nullptr, int est = bsa::kEstMean,
+                      const bsa::HeadMap* map = nullptr) {
   int need = 0;
   bsa_status s = check_params(p, mode, param, &need);
   if (s != BSA_OK) return s;
@@ -232,6 +233,7 @@ bsa_status run_select(const bsa_plan_s* p, const float* qc, const float* kc, bsa
   a.qc = qc; a.kc = kc; a.idx = idx; a.cnt = cnt; a.scores = scores; a.kmax = kmax;
   a.mode = (int)mode;
   a.est = est;
+  if (map) a.map = *map;
   a.scale = (float)(1.0 / std::sqrt((double)p->g.D));
   for (int h = 0; h < p->g.Hd; ++h)
     a.param[h] = mode == BSA_TOPK ? (double)k_for_density(param[h], p->g.nb) : param[h];
@@ -247,6 +249,7 @@ bsa_status run_select(const bsa_plan_s* p, const float* qc, const float* kc, bsa
       ia.scores = intra_scores;
       ia.bits = bits;
       ia.mode = uo->intra_mode;
+      if (map) ia.map = *map;
       for (int h = 0; h < p->g.Hd; ++h) ia.param[h] = uo->intra_param[h];
       cudaError_t e = bsa::launch_intra_select(p->g, ia, st);
       if (e != cudaSuccess) return cuda_fail(e, "intra select kernel");
@@ -266,6 +269,7 @@ bsa_status run_attention(const bsa_plan_s* p, const void* q, const void* k, cons
   if (p->g.nb > 0 && (!idx || !cnt)) return fail(BSA_ERR_INVALID_ARG, "NULL index list");
   if (kmax < 1) return fail(BSA_ERR_INVALID_ARG, "kmax must be >= 1");
   bsa::AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
   a.q = q; a.k = k; a.v = v; a.o = o; a.idx = idx; a.cnt = cnt; a.masks = p->d_masks;
   a.status = dev_status ? dev_status : p->d_status;
   a.kmax = kmax;
@@ -290,10 +294,12 @@ bsa_status run_attention(const bsa_plan_s* p, const void* q, const void* k, cons
 // Summaries straight from the original layout: centroids (MEAN) or (max,
 // min) boxes (DSA, DSA2) of Q and K, optionally with the SICS of the K blocks.
 bsa_status run_centroids(const bsa_plan_s* p, const void* q, const void* k, float* qc, float* kc,
-                         cudaStream_t st, float* k_sics = nullptr, bool boxes = false) {
+                         cudaStream_t st, float* k_sics = nullptr, bool boxes = false,
+                         const bsa::HeadMap* map = nullptr) {
   // Only the requested tensors are read.
   bsa::GatherArgs ga;
   std::memset(&ga, 0, sizeof(ga));
+  if (map) ga.map = *map;
   if (qc) {
     ga.src[ga.ntensors] = q;
     (boxes ? ga.box : ga.cent)[ga.ntensors] = qc;
@@ -313,7 +319,8 @@ bsa_status run_centroids(const bsa_plan_s* p, const void* q, const void* k, floa
 // Attention on the original layout, one launch per batch element.
 bsa_status run_attention_orig(const bsa_plan_s* p, const void* q, const void* k, const void* v,
                               const int32_t* idx, const int32_t* cnt, int kmax, void* o,
-                              int32_t* dev_status, cudaStream_t st) {
+                              int32_t* dev_status, cudaStream_t st,
+                              const bsa::HeadMap* map = nullptr) {
   if (p->attn_path != 1)
     return fail(BSA_ERR_UNSUPPORTED, "attention on the original layout needs a bf16 plan with 128-token blocks");
   if (!q || !k || !v || !o) return fail(BSA_ERR_INVALID_ARG, "NULL tensor pointer");
@@ -326,6 +333,14 @@ bsa_status run_attention_orig(const bsa_plan_s* p, const void* q, const void* k,
   g1.B = 1;
   bsa_status s;
   for (int b = 0; b < p->g.B; ++b) {
+    // the heads of this batch element that the map selects (all without one)
+    bsa::HeadMap hm;
+    std::memset(&hm, 0, sizeof(hm));
+    if (map && map->n) {
+      for (int x = 0; x < map->n; ++x)
+        if (map->bh[x] / p->g.Hd == b) hm.bh[hm.n++] = (uint8_t)(map->bh[x] % p->g.Hd);
+      if (hm.n == 0) continue;
+    }
     bsa::TileMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     const char* qb = reinterpret_cast<const char*>(q) + b * per_batch;
@@ -335,6 +350,8 @@ bsa_status run_attention_orig(const bsa_plan_s* p, const void* q, const void* k,
     if ((s = make_orig_maps(&maps.k, &maps.kt, kb, p->g)) != BSA_OK) return s;
     if ((s = make_orig_maps(&maps.v, &maps.vt, vb, p->g)) != BSA_OK) return s;
     bsa::AttnArgs a;
+    std::memset(&a, 0, sizeof(a));
+  std::memset(&a, 0, sizeof(a));
     a.q = qb; a.k = kb; a.v = vb;
     a.o = reinterpret_cast<char*>(o) + b * per_batch;
     a.idx = idx + (size_t)b * p->g.Hd * p->g.nb * kmax;
@@ -344,6 +361,7 @@ bsa_status run_attention_orig(const bsa_plan_s* p, const void* q, const void* k,
     a.kmax = kmax;
     a.scale = (float)(1.0 / std::sqrt((double)p->g.D));
     a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->g.D));
+    a.map = hm;
     cudaError_t e = bsa::launch_attn_tc_orig(g1, a, maps, st);
     if (e != cudaSuccess) return cuda_fail(e, "attention kernel");
   }
@@ -462,6 +480,39 @@ bsa_status forward_impl(bsa_plan_t p, const void* q, const void* k, const void* 
     return s;
   if ((s = run_attention(p, q_blk, k_blk, v_blk, idx, cnt, kmax, o_blk, dev_status, st)) != BSA_OK) return s;
   return bsa_unpermute(p, o_blk, o, stream);
+}
+
+// Workspace of one scheme group of bsa_forward_grouped: its centroids, its
+// lists and, with an intra part, its K-block SICS and bit sets.
+size_t group_ws_bytes(const bsa_plan_s* p, int kmax, bool intra) {
+  size_t w = 2 * round256(cent_bytes(p)) +
+             round256((size_t)p->g.B * p->g.Hd * p->g.nb * kmax * sizeof(int32_t)) +
+             round256((size_t)p->g.B * p->g.Hd * p->g.nb * sizeof(int32_t));
+  if (intra) w += round256(sics_bytes(p)) + round256(bits_bytes(p));
+  return w;
+}
+
+// Checks that the candidate plans describe the same problem (only the block
+// shape differs), run on the tensor-core path, and that a head map fits.
+bsa_status check_group_plans(const bsa_plan_t* plans, int n_plans) {
+  if (plans == nullptr) return fail(BSA_ERR_INVALID_ARG, "NULL plan array");
+  if (n_plans < 1 || n_plans > bsa::kMaxSchemes)
+    return fail(BSA_ERR_INVALID_ARG, "n_plans = %d, must be in [1, %d]", n_plans, bsa::kMaxSchemes);
+  for (int c = 0; c < n_plans; ++c) {
+    bsa_status s = check_plan(plans[c]);
+    if (s != BSA_OK) return s;
+    const Geo& g = plans[c]->g;
+    const Geo& g0 = plans[0]->g;
+    if (g.B != g0.B || g.T != g0.T || g.H != g0.H || g.W != g0.W || g.Hd != g0.Hd ||
+        g.D != g0.D || g.n_text != g0.n_text || plans[c]->dtype != plans[0]->dtype)
+      return fail(BSA_ERR_INVALID_ARG,
+                  "plan %d differs from plan 0 in more than the block shape", c);
+    if (plans[c]->attn_path != 1)
+      return fail(BSA_ERR_UNSUPPORTED, "grouped forward needs bf16 plans with 128-token blocks");
+  }
+  if ((long long)plans[0]->g.B * plans[0]->g.Hd > BSA_MAX_HEADS)
+    return fail(BSA_ERR_UNSUPPORTED, "grouped forward needs batch * heads <= %d", BSA_MAX_HEADS);
+  return BSA_OK;
 }
 
 }  // namespace
@@ -832,6 +883,91 @@ bsa_status bsa_aggregation_scores(const bsa_plan_t* plans, int n_plans, const vo
   if ((long long)g0.B * g0.Hd == 0) return BSA_OK;
   cudaError_t e = bsa::launch_sics_schemes(a, plans[0]->dtype == BSA_BF16, (cudaStream_t)stream);
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "SICS kernel");
+}
+
+bsa_status bsa_grouped_workspace_size(const bsa_plan_t* plans, int n_plans, const int* kmax_per_plan,
+                                      const bsa_mask_union_t* u, size_t* forward_ws) {
+  bsa_status s = check_group_plans(plans, n_plans);
+  if (s != BSA_OK) return s;
+  if (kmax_per_plan == nullptr) return fail(BSA_ERR_INVALID_ARG, "NULL kmax_per_plan");
+  size_t total = 0;
+  for (int c = 0; c < n_plans; ++c) {
+    UnionOpts uo;
+    int extra = 0;
+    if ((s = check_union(plans[c], u, &uo, &extra)) != BSA_OK) return s;
+    if (kmax_per_plan[c] < 1) return fail(BSA_ERR_INVALID_ARG, "kmax of plan %d must be >= 1", c);
+    total += group_ws_bytes(plans[c], kmax_per_plan[c], uo.intra);
+  }
+  if (forward_ws) *forward_ws = total;
+  return BSA_OK;
+}
+
+bsa_status bsa_forward_grouped(const bsa_plan_t* plans, int n_plans, const int32_t* head_plan,
+                               const void* q, const void* k, const void* v, bsa_select_mode mode,
+                               const double* param, const bsa_mask_union_t* u,
+                               const int* kmax_per_plan, void* o, int32_t* const* idx_out,
+                               int32_t* const* cnt_out, void* ws, size_t ws_bytes,
+                               int32_t* dev_status, void* stream) {
+  size_t need_ws = 0;
+  bsa_status s = bsa_grouped_workspace_size(plans, n_plans, kmax_per_plan, u, &need_ws);
+  if (s != BSA_OK) return s;
+  const Geo& g0 = plans[0]->g;
+  const int BH = g0.B * g0.Hd;
+  if (head_plan == nullptr) return fail(BSA_ERR_INVALID_ARG, "NULL head_plan");
+  for (int bh = 0; bh < BH; ++bh)
+    if (head_plan[bh] < 0 || head_plan[bh] >= n_plans)
+      return fail(BSA_ERR_INVALID_ARG, "head_plan[%d] = %d is not a plan index", bh, head_plan[bh]);
+  for (int c = 0; c < n_plans; ++c) {
+    int need = 0;
+    if ((s = union_kmax(plans[c], mode, param, u, &need)) != BSA_OK) return s;
+    if (kmax_per_plan[c] < need)
+      return fail(BSA_ERR_INVALID_ARG, "kmax %d of plan %d is below the %d entries a list can need",
+                  kmax_per_plan[c], c, need);
+  }
+  if (!q || !k || !v || !o) return fail(BSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if (ws == nullptr || ws_bytes < need_ws)
+    return fail(BSA_ERR_WORKSPACE, "grouped forward needs %zu bytes of workspace, got %zu", need_ws, ws_bytes);
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(BSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  char* w = reinterpret_cast<char*>(ws);
+  for (int c = 0; c < n_plans; ++c) {
+    const bsa_plan_s* p = plans[c];
+    const int kmax = kmax_per_plan[c];
+    UnionOpts uo;
+    int extra = 0;
+    check_union(p, u, &uo, &extra);
+    char* base = w;
+    w += group_ws_bytes(p, kmax, uo.intra);
+    bsa::HeadMap map;
+    std::memset(&map, 0, sizeof(map));
+    for (int bh = 0; bh < BH; ++bh)
+      if (head_plan[bh] == c) map.bh[map.n++] = (uint8_t)bh;
+    if (map.n == 0) continue;
+    const size_t cb = round256(cent_bytes(p));
+    float* qc = reinterpret_cast<float*>(base); base += cb;
+    float* kc = reinterpret_cast<float*>(base); base += cb;
+    int32_t* idx = reinterpret_cast<int32_t*>(base);
+    base += round256((size_t)p->g.B * p->g.Hd * p->g.nb * kmax * sizeof(int32_t));
+    int32_t* cnt = reinterpret_cast<int32_t*>(base);
+    base += round256((size_t)p->g.B * p->g.Hd * p->g.nb * sizeof(int32_t));
+    float* k_sics = nullptr;
+    uint32_t* bits = nullptr;
+    if (uo.intra) {
+      k_sics = reinterpret_cast<float*>(base); base += round256(sics_bytes(p));
+      bits = reinterpret_cast<uint32_t*>(base);
+    }
+    if (idx_out && idx_out[c]) idx = idx_out[c];
+    if (cnt_out && cnt_out[c]) cnt = cnt_out[c];
+    if ((s = run_centroids(p, q, k, qc, kc, st, k_sics, false, &map)) != BSA_OK) return s;
+    if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st, u ? &uo : nullptr,
+                        k_sics, bits, bsa::kEstMean, &map)) != BSA_OK)
+      return s;
+    if ((s = run_attention_orig(p, q, k, v, idx, cnt, kmax, o, dev_status, st, &map)) != BSA_OK)
+      return s;
+  }
+  return BSA_OK;
 }
 
 bsa_status bsa_check_status(bsa_plan_t p, void* stream) {

@@ -27,20 +27,23 @@ namespace bsa {
 
 // Tile order: text query tiles first (they have the longest lists), then the
 // video tiles, head-major so that one head's K/V stays resident in L2.
-__device__ __forceinline__ void decode_tile(const Geo& g, int L, int& b, int& h, int& i) {
-  const int n_text_tiles = g.B * g.Hd * g.nb_text;
+// The (batch, head) pairs come from the launch's head map (all of them when
+// it is empty).
+__device__ __forceinline__ void decode_tile(const Geo& g, const HeadMap& m, int L, int& b, int& h,
+                                            int& i) {
+  const int n_text_tiles = map_count(m, g.B * g.Hd) * g.nb_text;
+  int slot;
   if (L < n_text_tiles) {
     i = g.nb + L % g.nb_text;
-    const int bh = L / g.nb_text;
-    h = bh % g.Hd;
-    b = bh / g.Hd;
+    slot = L / g.nb_text;
   } else {
     L -= n_text_tiles;
     i = L % g.nb;
-    const int bh = L / g.nb;
-    h = bh % g.Hd;
-    b = bh / g.Hd;
+    slot = L / g.nb;
   }
+  const int bh = map_bh(m, slot);
+  h = bh % g.Hd;
+  b = bh / g.Hd;
 }
 
 __device__ __forceinline__ void set_status(int32_t* st, int code) {
@@ -90,7 +93,7 @@ __global__ void __launch_bounds__(kSimtWarps * 32) attn_simt_kernel(Geo g, AttnA
   constexpr int DL = D / 32;  // elements of a row per lane
   __shared__ float s_q[kSimtWarps][D];
   int b, h, i;
-  decode_tile(g, blockIdx.x, b, h, i);
+  decode_tile(g, a.map, blockIdx.x, b, h, i);
   const long long bh = (long long)b * g.Hd + h;
   const int nbk = g.nb + g.nb_text;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -156,7 +159,7 @@ __global__ void __launch_bounds__(kSimtWarps * 32) attn_simt_kernel(Geo g, AttnA
 }
 
 cudaError_t launch_attn_simt(const Geo& g, bool is_bf16, const AttnArgs& a, cudaStream_t st) {
-  const int tiles = g.B * g.Hd * (g.nb + g.nb_text);
+  const int tiles = map_count(a.map, g.B * g.Hd) * (g.nb + g.nb_text);
   if (tiles == 0) return cudaSuccess;
   if (is_bf16) {
     if (g.D == 128) attn_simt_kernel<__nv_bfloat16, 128><<<tiles, kSimtWarps * 32, 0, st>>>(g, a);
@@ -286,7 +289,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nbk = g.nb + g.nb_text;
-  const int n_tiles = g.B * g.Hd * nbk;
+  const int n_tiles = map_count(a.map, g.B * g.Hd) * nbk;
 
   // The two query tiles of this CTA (held in scalars: a runtime-indexed array
   // would live in local memory).
@@ -295,11 +298,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   {
     int b, h, i;
     if (2 * (int)blockIdx.x < n_tiles) {
-      decode_tile(g, 2 * blockIdx.x, b, h, i);
+      decode_tile(g, a.map, 2 * blockIdx.x, b, h, i);
       i0 = i; bh0 = (long long)b * g.Hd + h; n0 = list_length(g, a, bh0, i);
     }
     if (2 * (int)blockIdx.x + 1 < n_tiles) {
-      decode_tile(g, 2 * blockIdx.x + 1, b, h, i);
+      decode_tile(g, a.map, 2 * blockIdx.x + 1, b, h, i);
       i1 = i; bh1 = (long long)b * g.Hd + h; n1 = list_length(g, a, bh1, i);
     }
   }
@@ -581,7 +584,7 @@ static cudaError_t launch_tc_t(const Geo& g, const AttnArgs& a, const TileMaps& 
 
 // Blocked layout in and out (bsa_attention).
 cudaError_t launch_attn_tc(const Geo& g, const AttnArgs& a, const TileMaps& maps, cudaStream_t st) {
-  const int tiles = g.B * g.Hd * (g.nb + g.nb_text);
+  const int tiles = map_count(a.map, g.B * g.Hd) * (g.nb + g.nb_text);
   if (tiles == 0) return cudaSuccess;
   const int ctas = (tiles + 1) / 2;
   return g.D == 128 ? launch_tc_t<128, false>(g, a, maps, ctas, st)
@@ -592,7 +595,7 @@ cudaError_t launch_attn_tc(const Geo& g, const AttnArgs& a, const TileMaps& maps
 // transform and its inverse happen inside the loads and the epilogue.
 cudaError_t launch_attn_tc_orig(const Geo& g, const AttnArgs& a, const TileMaps& maps,
                                 cudaStream_t st) {
-  const int tiles = g.Hd * (g.nb + g.nb_text);
+  const int tiles = map_count(a.map, g.Hd) * (g.nb + g.nb_text);
   if (tiles == 0 || g.B != 1) return g.B != 1 ? cudaErrorInvalidValue : cudaSuccess;
   const int ctas = (tiles + 1) / 2;
   return g.D == 128 ? launch_tc_t<128, true>(g, a, maps, ctas, st)

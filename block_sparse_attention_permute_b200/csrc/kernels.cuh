@@ -5,6 +5,16 @@
 
 namespace bsa {
 
+// The (batch, head) pairs one launch covers: n = 0 means all B * Hd pairs in
+// order; otherwise the pairs bh[0..n), bh = b * Hd + h (B * Hd <= 256).  This
+// is how heads that share a blocking scheme are grouped into one launch.
+struct HeadMap {
+  int n;
+  uint8_t bh[BSA_MAX_HEADS];
+};
+__host__ __device__ __forceinline__ int map_count(const HeadMap& m, int all) { return m.n ? m.n : all; }
+__host__ __device__ __forceinline__ int map_bh(const HeadMap& m, int x) { return m.n ? (int)m.bh[x] : x; }
+
 struct GatherArgs {
   const void* src[3];
   void* dst[3];      // unused in kPool
@@ -12,6 +22,7 @@ struct GatherArgs {
   float* sics[3];    // optional SICS outputs [B, Hd, nb] (kPermute, kPool, kPoolOrig)
   float* box[3];     // optional box summaries [B, Hd, nb, D, 2] = (max, min) (same modes)
   int ntensors;
+  HeadMap map;
 };
 
 // Aggregation evaluation of up to kMaxSchemes candidate blocking schemes of
@@ -47,6 +58,7 @@ struct SelectArgs {
   int win_left, win_right;      // j in [i - left, i + right]; < 0 = unbounded; both < 0 = none
   long long sink_tokens;        // blocks holding any of the first sink_tokens tokens
   const uint32_t* intra_bits;   // [B, Hd, nbw] selected key blocks, or null
+  HeadMap map;
 };
 
 // Selection on per-key-block intra scores (one warp per (b, h)).
@@ -55,6 +67,7 @@ struct IntraArgs {
   uint32_t* bits;               // [B, Hd, nbw], nbw = ceil(nb / 32)
   int mode;                     // 0 top-k, 1 top-p
   double param[BSA_MAX_HEADS];  // k (held in a double) or tau per head; <= 0 = none
+  HeadMap map;
 };
 
 struct AttnArgs {
@@ -69,6 +82,7 @@ struct AttnArgs {
   int kmax;
   float scale;            // 1/sqrt(D)
   float scale_log2;       // log2(e)/sqrt(D)
+  HeadMap map;
 };
 
 // TMA tensor maps of one attention launch: q/k/v cover the blocked tensors

@@ -67,7 +67,7 @@ __device__ __forceinline__ void to_float(const uint4& v, float* f) {
 // rows is the r of the online form (Eq. (5)); squaring it once at the end
 // instead of accumulating the cross terms keeps every term of the fp32 sum
 // non-negative.
-template <typename T, int D, int MODE>
+template <typename T, int D, int MODE, bool EXTRAS>
 __device__ __forceinline__ void gather_block(const Geo& g, const void* src_ptr, void* dst_ptr,
                                              float* cent_ptr, float* sics_ptr, float* box_ptr,
                                              int j, int h, int b) {
@@ -86,8 +86,10 @@ __device__ __forceinline__ void gather_block(const Geo& g, const void* src_ptr, 
   const long long blk_row0 = (long long)(b * g.Hd + h) * g.npad_tot + (long long)j * g.bs;
   const long long tok_base = (long long)b * g.n_tot;
   float* cent = (MODE != kUnpermute && j < g.nb) ? cent_ptr : nullptr;
-  float* sics = (MODE != kUnpermute && j < g.nb) ? sics_ptr : nullptr;
-  float* box = (MODE != kUnpermute && j < g.nb) ? box_ptr : nullptr;
+  // SICS and box outputs exist only in the EXTRAS instances, which keeps
+  // the plain copy / centroid instances lean (registers, occupancy).
+  float* sics = (EXTRAS && MODE != kUnpermute && j < g.nb) ? sics_ptr : nullptr;
+  float* box = (EXTRAS && MODE != kUnpermute && j < g.nb) ? box_ptr : nullptr;
   float acc[E], racc[E], vmax[E], vmin[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
@@ -119,7 +121,7 @@ __device__ __forceinline__ void gather_block(const Geo& g, const void* src_ptr, 
       if (MODE == kPermute && tok[u] >= -1) dst[(blk_row0 + s) * V + vec] = buf[u];
       if (MODE == kUnpermute && tok[u] >= 0) dst[((tok_base + tok[u]) * g.Hd + h) * V + vec] = buf[u];
       if (MODE != kUnpermute && cent != nullptr && tok[u] >= 0) accumulate_vec<T>(acc, buf[u]);
-      if (MODE != kUnpermute && box != nullptr && tok[u] >= 0) {
+      if (EXTRAS && MODE != kUnpermute && box != nullptr && tok[u] >= 0) {
         float f[E];
         to_float<T>(buf[u], f);
 #pragma unroll
@@ -128,7 +130,7 @@ __device__ __forceinline__ void gather_block(const Geo& g, const void* src_ptr, 
           vmin[e] = fminf(vmin[e], f[e]);
         }
       }
-      if (MODE != kUnpermute && sics != nullptr) {
+      if (EXTRAS && MODE != kUnpermute && sics != nullptr) {
         // Every lane takes part (pad and out-of-range rows hold zeros): the V
         // lanes of one row are an aligned group of the warp.
         float f[E], ss = 0.f;
@@ -156,7 +158,7 @@ __device__ __forceinline__ void gather_block(const Geo& g, const void* src_ptr, 
     }
   }
 
-  if (MODE != kUnpermute && box != nullptr) {
+  if (EXTRAS && MODE != kUnpermute && box != nullptr) {
     // per dimension: max, then min, over the R row groups (exact in fp32)
     float* out = box + ((long long)(b * g.Hd + h) * g.nb + j) * D * 2;
 #pragma unroll
@@ -174,7 +176,7 @@ __device__ __forceinline__ void gather_block(const Geo& g, const void* src_ptr, 
     }
   }
 
-  if (MODE != kUnpermute && sics != nullptr) {
+  if (EXTRAS && MODE != kUnpermute && sics != nullptr) {
     __syncthreads();  // s_red is reused after the centroid reduction
 #pragma unroll
     for (int e = 0; e < E; ++e) s_red[row0 * D + vec * E + e] = racc[e];
@@ -197,18 +199,18 @@ __device__ __forceinline__ void gather_block(const Geo& g, const void* src_ptr, 
   }
 }
 
-template <typename T, int D, int MODE>
+template <typename T, int D, int MODE, bool EXTRAS>
 __global__ void __launch_bounds__(kGatherThreads) gather_kernel(Geo g, GatherArgs a) {
   // Constant-index reads of the pointer arrays (a dynamic index would copy
   // the argument block to local memory).
-  const int t = blockIdx.z % a.ntensors;
+  const int t = a.map.n ? (int)blockIdx.z : (int)(blockIdx.z % a.ntensors);
+  const int bh = a.map.n ? (int)a.map.bh[blockIdx.y] : (int)(blockIdx.z / a.ntensors) * g.Hd + (int)blockIdx.y;
   const void* src = t == 0 ? a.src[0] : t == 1 ? a.src[1] : a.src[2];
   void* dst = t == 0 ? a.dst[0] : t == 1 ? a.dst[1] : a.dst[2];
   float* cent = t == 0 ? a.cent[0] : t == 1 ? a.cent[1] : a.cent[2];
   float* sics = t == 0 ? a.sics[0] : t == 1 ? a.sics[1] : a.sics[2];
   float* box = t == 0 ? a.box[0] : t == 1 ? a.box[1] : a.box[2];
-  gather_block<T, D, MODE>(g, src, dst, cent, sics, box, blockIdx.x, blockIdx.y,
-                           blockIdx.z / a.ntensors);
+  gather_block<T, D, MODE, EXTRAS>(g, src, dst, cent, sics, box, blockIdx.x, bh % g.Hd, bh / g.Hd);
 }
 
 // Aggregation evaluation (SPADE §3.2): SICS of every block of every candidate
@@ -370,11 +372,20 @@ __global__ void __launch_bounds__(128) aggregate_kernel(SchemeArgs s, int BH) {
 template <typename T, int MODE>
 static cudaError_t launch_gather_t(const Geo& g, const GatherArgs& a, int nblocks,
                                    cudaStream_t st) {
-  dim3 grid(nblocks, g.Hd, g.B * a.ntensors);
-  if (g.D == 128)
-    gather_kernel<T, 128, MODE><<<grid, kGatherThreads, 0, st>>>(g, a);
-  else
-    gather_kernel<T, 64, MODE><<<grid, kGatherThreads, 0, st>>>(g, a);
+  dim3 grid(nblocks, a.map.n ? a.map.n : g.Hd, a.map.n ? a.ntensors : g.B * a.ntensors);
+  bool extras = false;
+  for (int t = 0; t < a.ntensors; ++t) extras = extras || a.sics[t] != nullptr || a.box[t] != nullptr;
+  if (MODE != kUnpermute && extras) {
+    if (g.D == 128)
+      gather_kernel<T, 128, MODE, true><<<grid, kGatherThreads, 0, st>>>(g, a);
+    else
+      gather_kernel<T, 64, MODE, true><<<grid, kGatherThreads, 0, st>>>(g, a);
+  } else {
+    if (g.D == 128)
+      gather_kernel<T, 128, MODE, false><<<grid, kGatherThreads, 0, st>>>(g, a);
+    else
+      gather_kernel<T, 64, MODE, false><<<grid, kGatherThreads, 0, st>>>(g, a);
+  }
   return cudaGetLastError();
 }
 

@@ -175,13 +175,14 @@ __device__ __forceinline__ float box_max_product(float aM, float am, float bM, f
 // D = length of the stored summary vectors (head_dim for MEAN, 2 * head_dim
 // for the (max, min) boxes of DSA and DSA2).
 template <int D, int EST>
-__global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, SelectArgs a) {
+__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(Geo g, SelectArgs a) {
   extern __shared__ __align__(16) float sm[];
   float* qs = sm;                                   // [kSelRows][D]
   float* ks = qs + kSelRows * D;                    // [kSelKeys][kSelDChunk+4]
   float* sc = ks + kSelKeys * (kSelDChunk + 4);     // [kSelRows][nb]
   const int nb = g.nb;
-  const int h = blockIdx.y, b = blockIdx.z;
+  const int bhi = map_bh(a.map, (int)blockIdx.z * g.Hd + (int)blockIdx.y);
+  const int h = bhi % g.Hd, b = bhi / g.Hd;
   const long long bh = (long long)b * g.Hd + h;
   const int i0 = blockIdx.x * kSelRows;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -322,8 +323,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, SelectArgs a
 constexpr int kIntraWarps = 4;
 
 __global__ void __launch_bounds__(kIntraWarps * 32) intra_select_kernel(Geo g, IntraArgs a) {
-  const int bh = blockIdx.x * kIntraWarps + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (bh >= g.B * g.Hd) return;
+  const int slot = blockIdx.x * kIntraWarps + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (slot >= map_count(a.map, g.B * g.Hd)) return;
+  const int bh = map_bh(a.map, slot);
   const int nb = g.nb, nbw = (nb + 31) / 32, h = bh % g.Hd;
   const float* row = a.scores + (long long)bh * nb;
   uint32_t* bits = a.bits + (long long)bh * nbw;
@@ -352,7 +354,7 @@ __global__ void __launch_bounds__(kIntraWarps * 32) intra_select_kernel(Geo g, I
 }
 
 cudaError_t launch_intra_select(const Geo& g, const IntraArgs& a, cudaStream_t st) {
-  const int BH = g.B * g.Hd;
+  const int BH = map_count(a.map, g.B * g.Hd);
   if (BH == 0 || g.nb == 0) return cudaSuccess;
   intra_select_kernel<<<(BH + kIntraWarps - 1) / kIntraWarps, kIntraWarps * 32, 0, st>>>(g, a);
   return cudaGetLastError();
@@ -361,7 +363,9 @@ cudaError_t launch_intra_select(const Geo& g, const IntraArgs& a, cudaStream_t s
 template <int D, int EST>
 static cudaError_t launch_select_t(const Geo& g, const SelectArgs& a, cudaStream_t st) {
   const size_t smem = select_smem_bytes(g.nb, D);
-  dim3 grid((g.nb + kSelRows - 1) / kSelRows, g.Hd, g.B);
+  // with a head map, y enumerates its pairs (z = 1) and the kernel reads
+  // map_bh(y); without one, y = h and z = b
+  dim3 grid((g.nb + kSelRows - 1) / kSelRows, a.map.n ? a.map.n : g.Hd, a.map.n ? 1 : g.B);
   cudaError_t e = cudaFuncSetAttribute(select_kernel<D, EST>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

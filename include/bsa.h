@@ -405,6 +405,52 @@ bsa_status bsa_forward_estimator(bsa_plan_t plan, const void* q, const void* k,
                                  size_t ws_bytes, int32_t* dev_status,
                                  void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Head grouping with per-head blocking schemes (SPADE §3.3 (2): "groups heads
+ * sharing a blocking scheme to increase per-launch work"; §3.2: each head
+ * takes its Selected Blocking Scheme).  The candidate plans describe one
+ * problem with different block shapes (as for bsa_aggregation_scores); each
+ * (b, h) is served by the plan head_plan[b * Hd + h] names — for instance the
+ * choice bsa_aggregation_scores returns, copied to the host.  The heads of
+ * one plan are one group: one centroid launch, one selection launch and one
+ * attention launch per batch element cover exactly those heads; the output
+ * rows of every head are written once. */
+
+/* bsa_grouped_workspace_size — workspace of bsa_forward_grouped: per plan its
+ * centroids, lists (kmax_per_plan[c] wide) and, with an intra part in u, its
+ * K-block SICS and bit sets. */
+bsa_status bsa_grouped_workspace_size(const bsa_plan_t* plans, int n_plans,
+                                      const int* kmax_per_plan,
+                                      const bsa_mask_union_t* u,
+                                      size_t* forward_ws);
+
+/* bsa_forward_grouped — bsa_forward_union with a blocking scheme per (b, h).
+ *   plans, n_plans  1..8 tensor-core plans (bf16, 128-token blocks) on the
+ *                   current device that agree in everything but the block
+ *                   shape; batch * heads <= 256
+ *   head_plan       host [B * Hd] int32: plan index of each (b, h)
+ *   q, k, v, o      [B, Ntot, Hd, D] original order
+ *   mode, param_per_head, u   selection and mask union, as bsa_forward_union
+ *                   (per-head parameters apply whatever the head's plan)
+ *   kmax_per_plan   host [n_plans]: list width per plan (>= the plan's
+ *                   bsa_kmax_for_union)
+ *   idx_out, cnt_out  host arrays of n_plans device pointers to
+ *                   [B, Hd, nb_c, kmax_c] / [B, Hd, nb_c] lists, or NULL
+ *                   (either array or entry); only the (b, h) of plan c are
+ *                   written in plan c's lists
+ *   ws, ws_bytes    >= bsa_grouped_workspace_size
+ * BSA_ERR_UNSUPPORTED for plans off the tensor-core path. */
+bsa_status bsa_forward_grouped(const bsa_plan_t* plans, int n_plans,
+                               const int32_t* head_plan, const void* q,
+                               const void* k, const void* v,
+                               bsa_select_mode mode,
+                               const double* param_per_head,
+                               const bsa_mask_union_t* u,
+                               const int* kmax_per_plan, void* o,
+                               int32_t* const* idx_out, int32_t* const* cnt_out,
+                               void* ws, size_t ws_bytes, int32_t* dev_status,
+                               void* stream);
+
 /* bsa_check_status — synchronise `stream`, read and clear the plan-owned
  * status word; returns BSA_OK or the recorded error. */
 bsa_status bsa_check_status(bsa_plan_t plan, void* stream);
