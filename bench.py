@@ -467,12 +467,20 @@ def run_ours(args, rank, world, local):
     qc, kc = (torch.empty(plan.cent_shape, dtype=torch.float32, device=dev) for _ in range(2))
     S = lambda: bsa._stream(dev)
     if plan.info.attn_path == 1:
-        # what bsa_forward runs on this plan: the layout transform is fused into the attention
+        # what bsa_forward runs on this plan: the layout transform is fused into
+        # the attention, whose query tiles are paired by shared key blocks
+        pz = ctypes.c_size_t()
+        bsa._check(L.bsa_pair_workspace_size(plan._h, kmax, ctypes.byref(pz)))
+        pws = torch.empty(pz.value, dtype=torch.uint8, device=dev)
         fused = time_phases(
-            ["centroids", "select", "attention"],
+            ["centroids", "select", "pairing", "attention", "attention_unpaired"],
             [lambda: L.bsa_centroids(plan._h, P(qd), P(kd), P(qc), P(kc), S()),
              lambda: L.bsa_select_centroids(plan._h, P(qc), P(kc), w.mode, params, kmax, P(idx),
                                             P(cnt), None, S()),
+             lambda: L.bsa_pair_tiles(plan._h, P(idx), P(cnt), kmax, P(pws), pws.numel(), S()),
+             lambda: L.bsa_attention_paired(plan._h, P(qd), P(kd), P(vd), P(idx), P(cnt), kmax,
+                                            P(pws), pws.numel(), P(out), None, S()),
+             # the same lists without pairing, for comparison (not part of the step)
              lambda: L.bsa_attention_orig(plan._h, P(qd), P(kd), P(vd), P(idx), P(cnt), kmax, P(out),
                                           None, S())])
     else:
@@ -609,13 +617,14 @@ def run_ours(args, rank, world, local):
         "attn_tflops": round(attn_tf, 2),
         "attn_frac_of_peak": round(attn_tf / peak_tf, 4),
         "permute_select_share_of_attn": round(
-            (phase_ms.get("centroids", phase_ms.get("permute", 0.0)) + phase_ms["select"])
-            / phase_ms["attention"], 4),
+            (phase_ms.get("centroids", phase_ms.get("permute", 0.0)) + phase_ms["select"]
+             + phase_ms.get("pairing", 0.0)) / phase_ms["attention"], 4),
         "permute_select_share_of_attn_unfused": round(
             (unfused["permute"] + unfused["select"]) / unfused["attention"], 4),
         "roofline": {
             "bound": "tensor",
-            "kernel": "attn_tc_kernel<128, original layout>" if plan.info.attn_path == 1 else "attn_simt_kernel",
+            "kernel": "attn_tc_kernel<128, original layout, paired tiles>" if plan.info.attn_path == 1
+                      else "attn_simt_kernel",
             "achieved": round(attn_tf, 2),
             "peak": peak_tf,
             "peak_source": f"{peak_src} bf16_tflops_sustained (MEASURED_PEAKS.json)",
@@ -636,7 +645,8 @@ def run_ours(args, rank, world, local):
         "scheme_generation": dict(scheme, share_of_attn=round(scheme["ms"] / phase_ms["attention"], 4),
                                   frac=round(scheme["achieved_gbs"] / hbm_gbs, 4),
                                   peak_gbs=hbm_gbs, bound="hbm"),
-        "gpu_launches": (3 if plan.info.attn_path == 1 else 4) * args.steps,
+        # tensor-core plans: centroids, select, 3 pairing kernels, attention
+        "gpu_launches": (6 if plan.info.attn_path == 1 else 4) * args.steps,
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -86,6 +86,9 @@ def load():
         "bsa_estimator_workspace_size": [P, I, I, P, ctypes.POINTER(Z)],
         "bsa_forward_estimator": [P, P, P, P, I, I, P, P, I, P, P, P, P, Z, P, P],
         "bsa_grouped_workspace_size": [P, I, P, P, ctypes.POINTER(Z)],
+        "bsa_pair_workspace_size": [P, I, ctypes.POINTER(Z)],
+        "bsa_pair_tiles": [P, P, P, I, P, Z, P],
+        "bsa_attention_paired": [P, P, P, P, P, P, I, P, Z, P, P, P],
         "bsa_forward_grouped": [P, I, P, P, P, P, I, P, P, P, P, P, P, P, Z, P, P],
         "bsa_aggregation_scores": [P, I, P, P, P, P, P],
     }
@@ -238,6 +241,26 @@ class Plan:
         out = self._new((i.batch, i.heads, i.nb), torch.float32) if out is None else out
         self._check_tensor(out, (i.batch, i.heads, i.nb), torch.float32, "out")
         _check(load().bsa_sics(self._h, _ptr(x), _ptr(out), _stream(self.device)))
+        return out
+
+    def pair_tiles(self, idx, cnt):
+        """bsa_pair_tiles: the pairing workspace (a uint8 tensor) for these lists."""
+        z = ctypes.c_size_t()
+        kmax = idx.shape[-1]
+        _check(load().bsa_pair_workspace_size(self._h, kmax, ctypes.byref(z)))
+        ws = self._new((max(z.value, 1),), torch.uint8)
+        _check(load().bsa_pair_tiles(self._h, _ptr(idx), _ptr(cnt), kmax, _ptr(ws), ws.numel(),
+                                     _stream(self.device)))
+        return ws
+
+    def attention_paired(self, q, k, v, idx, cnt, ws, out=None, dev_status=None):
+        """bsa_attention_paired on the schedule of pair_tiles(idx, cnt)."""
+        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+            self._check_tensor(t, self.orig_shape, name=n)
+        out = self._new(self.orig_shape) if out is None else out
+        _check(load().bsa_attention_paired(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt),
+                                           idx.shape[-1], _ptr(ws), ws.numel(), _ptr(out),
+                                           _ptr(dev_status), _stream(self.device)))
         return out
 
     def attention_orig(self, q, k, v, idx, cnt, out=None, dev_status=None):

@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libbsa.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
-SOURCES = ["permute.cu", "select.cu", "attn.cu", "api.cu", "select_static.cu"]
+SOURCES = ["permute.cu", "select.cu", "pair.cu", "attn.cu", "api.cu", "select_static.cu"]
 HEADERS = ["common.cuh", "kernels.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

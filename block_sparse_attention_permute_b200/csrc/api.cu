@@ -317,10 +317,50 @@ bsa_status run_centroids(const bsa_plan_s* p, const void* q, const void* k, floa
 }
 
 // Attention on the original layout, one launch per batch element.
+// Query tiles per head paired for K/V sharing (pair.cu): text pairs, then
+// video pairs.
+int text_pairs(const Geo& g) { return (g.nb_text + 1) / 2; }
+int pairs_per_head(const Geo& g) { return text_pairs(g) + (g.nb + 1) / 2; }
+size_t pairing_bytes(const bsa_plan_s* p, int kmax) {
+  const size_t bh = (size_t)p->g.B * p->g.Hd, pph = pairs_per_head(p->g);
+  return round256(bsa::pair_scratch_bytes(p->g)) + round256(bh * pph * 4 * sizeof(int32_t)) +
+         round256(bh * pph * 2 * (size_t)kmax * sizeof(int32_t));
+}
+
+// Pairs the query tiles of the selected heads (scratch and schedule carved
+// from `w`, pairing_bytes long); on return *sched / *lists point at them.
+bsa_status run_pairing(const bsa_plan_s* p, const int32_t* idx, const int32_t* cnt, int kmax,
+                       char* w, int32_t** sched, int32_t** lists, cudaStream_t st,
+                       const bsa::HeadMap* map) {
+  const size_t bh = (size_t)p->g.B * p->g.Hd, pph = pairs_per_head(p->g);
+  const size_t nbw = (p->g.nb + 31) / 32;
+  bsa::PairArgs pa;
+  std::memset(&pa, 0, sizeof(pa));
+  pa.idx = idx;
+  pa.cnt = cnt;
+  pa.bits = reinterpret_cast<uint32_t*>(w);
+  pa.cand = reinterpret_cast<uint16_t*>(w + round256(bh * p->g.nb * nbw * sizeof(uint32_t)));
+  w += round256(bsa::pair_scratch_bytes(p->g));
+  pa.sched = reinterpret_cast<int32_t*>(w);
+  w += round256(bh * pph * 4 * sizeof(int32_t));
+  pa.lists = reinterpret_cast<int32_t*>(w);
+  pa.kmax = kmax;
+  pa.pairs_per_head = (int)pph;
+  pa.text_pairs = text_pairs(p->g);
+  if (map) pa.map = *map;
+  cudaError_t e = bsa::launch_pairing(p->g, pa, st);
+  if (e != cudaSuccess) return cuda_fail(e, "pairing kernels");
+  *sched = pa.sched;
+  *lists = pa.lists;
+  return BSA_OK;
+}
+
 bsa_status run_attention_orig(const bsa_plan_s* p, const void* q, const void* k, const void* v,
                               const int32_t* idx, const int32_t* cnt, int kmax, void* o,
                               int32_t* dev_status, cudaStream_t st,
-                              const bsa::HeadMap* map = nullptr) {
+                              const bsa::HeadMap* map = nullptr,
+                              const int32_t* pair_sched = nullptr,
+                              const int32_t* pair_lists = nullptr) {
   if (p->attn_path != 1)
     return fail(BSA_ERR_UNSUPPORTED, "attention on the original layout needs a bf16 plan with 128-token blocks");
   if (!q || !k || !v || !o) return fail(BSA_ERR_INVALID_ARG, "NULL tensor pointer");
@@ -362,6 +402,13 @@ bsa_status run_attention_orig(const bsa_plan_s* p, const void* q, const void* k,
     a.scale = (float)(1.0 / std::sqrt((double)p->g.D));
     a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->g.D));
     a.map = hm;
+    if (pair_sched != nullptr) {
+      const long long pph = pairs_per_head(p->g);
+      a.pair_sched = pair_sched + (long long)b * p->g.Hd * pph * 4;
+      a.pair_lists = pair_lists + (long long)b * p->g.Hd * pph * 2 * kmax;
+      a.pairs_per_head = (int)pph;
+      a.text_pairs = text_pairs(p->g);
+    }
     cudaError_t e = bsa::launch_attn_tc_orig(g1, a, maps, st);
     if (e != cudaSuccess) return cuda_fail(e, "attention kernel");
   }
@@ -374,14 +421,20 @@ bsa_status run_attention_orig(const bsa_plan_s* p, const void* q, const void* k,
 bsa_status run_forward_fused(const bsa_plan_s* p, const void* q, const void* k, const void* v,
                              bsa_select_mode mode, const double* param, int kmax, void* o,
                              int32_t* idx, int32_t* cnt, float* qc, float* kc,
-                             int32_t* dev_status, cudaStream_t st, const UnionOpts* uo = nullptr,
-                             float* k_sics = nullptr, uint32_t* bits = nullptr,
-                             int est = bsa::kEstMean) {
-  bsa_status s = run_centroids(p, q, k, qc, kc, st, k_sics, est != bsa::kEstMean);
+                             int32_t* dev_status, cudaStream_t st, const UnionOpts* uo,
+                             float* k_sics, uint32_t* bits, int est, char* pair_ws,
+                             const bsa::HeadMap* map = nullptr) {
+  bsa_status s = run_centroids(p, q, k, qc, kc, st, k_sics, est != bsa::kEstMean, map);
   if (s != BSA_OK) return s;
-  if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st, uo, k_sics, bits, est)) != BSA_OK)
+  if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st, uo, k_sics, bits, est,
+                      map)) != BSA_OK)
     return s;
-  return run_attention_orig(p, q, k, v, idx, cnt, kmax, o, dev_status, st);
+  int32_t* sched = nullptr;
+  int32_t* lists = nullptr;
+  if (pair_ws != nullptr &&
+      (s = run_pairing(p, idx, cnt, kmax, pair_ws, &sched, &lists, st, map)) != BSA_OK)
+    return s;
+  return run_attention_orig(p, q, k, v, idx, cnt, kmax, o, dev_status, st, map, sched, lists);
 }
 
 // kmax a list can need under the union: the inter bound plus the blocks the
@@ -454,7 +507,7 @@ bsa_status forward_impl(bsa_plan_t p, const void* q, const void* k, const void* 
   uint32_t* bits = nullptr;
   if (uo.intra) {
     k_sics = reinterpret_cast<float*>(w); w += round256(sics_bytes(p));
-    bits = reinterpret_cast<uint32_t*>(w);
+    bits = reinterpret_cast<uint32_t*>(w); w += round256(bits_bytes(p));
   }
   if (idx_out) idx = idx_out;
   if (cnt_out) cnt = cnt_out;
@@ -462,7 +515,7 @@ bsa_status forward_impl(bsa_plan_t p, const void* q, const void* k, const void* 
   const UnionOpts* up = u ? &uo : nullptr;
   if (p->attn_path == 1)
     return run_forward_fused(p, q, k, v, mode, param, kmax, o, idx, cnt, qc, kc, dev_status, st, up,
-                             k_sics, bits, est);
+                             k_sics, bits, est, w);
   bsa::GatherArgs a;
   std::memset(&a, 0, sizeof(a));
   a.src[0] = q; a.src[1] = k; a.src[2] = v;
@@ -489,7 +542,7 @@ size_t group_ws_bytes(const bsa_plan_s* p, int kmax, bool intra) {
              round256((size_t)p->g.B * p->g.Hd * p->g.nb * kmax * sizeof(int32_t)) +
              round256((size_t)p->g.B * p->g.Hd * p->g.nb * sizeof(int32_t));
   if (intra) w += round256(sics_bytes(p)) + round256(bits_bytes(p));
-  return w;
+  return w + pairing_bytes(p, kmax);
 }
 
 // Checks that the candidate plans describe the same problem (only the block
@@ -620,7 +673,11 @@ bsa_status bsa_workspace_size(bsa_plan_t p, int kmax, size_t* select_ws, size_t*
   if (select_ws) *select_ws = 2 * cent;
   // The tensor-core path fuses the layout transform into the attention loads;
   // the SIMT path stages blocked Q, K, V and O.
-  if (forward_ws) *forward_ws = (p->attn_path == 1 ? 0 : 4 * round256(blk_bytes(p))) + 2 * cent + lists;
+  // The SIMT path stages blocked Q, K, V and O; the tensor-core path fuses the
+  // layout transform into the attention loads and pairs the query tiles.
+  if (forward_ws)
+    *forward_ws = (p->attn_path == 1 ? pairing_bytes(p, kmax) : 4 * round256(blk_bytes(p))) +
+                  2 * cent + lists;
   return BSA_OK;
 }
 
@@ -956,18 +1013,56 @@ bsa_status bsa_forward_grouped(const bsa_plan_t* plans, int n_plans, const int32
     uint32_t* bits = nullptr;
     if (uo.intra) {
       k_sics = reinterpret_cast<float*>(base); base += round256(sics_bytes(p));
-      bits = reinterpret_cast<uint32_t*>(base);
+      bits = reinterpret_cast<uint32_t*>(base); base += round256(bits_bytes(p));
     }
     if (idx_out && idx_out[c]) idx = idx_out[c];
     if (cnt_out && cnt_out[c]) cnt = cnt_out[c];
-    if ((s = run_centroids(p, q, k, qc, kc, st, k_sics, false, &map)) != BSA_OK) return s;
-    if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st, u ? &uo : nullptr,
-                        k_sics, bits, bsa::kEstMean, &map)) != BSA_OK)
-      return s;
-    if ((s = run_attention_orig(p, q, k, v, idx, cnt, kmax, o, dev_status, st, &map)) != BSA_OK)
+    if ((s = run_forward_fused(p, q, k, v, mode, param, kmax, o, idx, cnt, qc, kc, dev_status, st,
+                               u ? &uo : nullptr, k_sics, bits, bsa::kEstMean, base, &map)) != BSA_OK)
       return s;
   }
   return BSA_OK;
+}
+
+bsa_status bsa_pair_workspace_size(bsa_plan_t p, int kmax, size_t* bytes) {
+  if (p == nullptr || bytes == nullptr) return fail(BSA_ERR_INVALID_ARG, "NULL plan or output");
+  if (kmax < 1) return fail(BSA_ERR_INVALID_ARG, "kmax must be >= 1");
+  *bytes = p->attn_path == 1 ? pairing_bytes(p, kmax) : 0;
+  return BSA_OK;
+}
+
+bsa_status bsa_pair_tiles(bsa_plan_t p, const int32_t* idx, const int32_t* cnt, int kmax, void* ws,
+                          size_t ws_bytes, void* stream) {
+  bsa_status s = check_plan(p);
+  if (s != BSA_OK) return s;
+  if (p->attn_path != 1)
+    return fail(BSA_ERR_UNSUPPORTED, "tile pairing serves bf16 plans with 128-token blocks");
+  if (kmax < 1) return fail(BSA_ERR_INVALID_ARG, "kmax must be >= 1");
+  if (p->g.nb > 0 && (!idx || !cnt)) return fail(BSA_ERR_INVALID_ARG, "NULL index list");
+  if (ws == nullptr || ws_bytes < pairing_bytes(p, kmax))
+    return fail(BSA_ERR_WORKSPACE, "pairing needs %zu bytes of workspace, got %zu",
+                pairing_bytes(p, kmax), ws_bytes);
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(BSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  int32_t* sched = nullptr;
+  int32_t* lists = nullptr;
+  return run_pairing(p, idx, cnt, kmax, reinterpret_cast<char*>(ws), &sched, &lists,
+                     (cudaStream_t)stream, nullptr);
+}
+
+bsa_status bsa_attention_paired(bsa_plan_t p, const void* q, const void* k, const void* v,
+                                const int32_t* idx, const int32_t* cnt, int kmax, const void* ws,
+                                size_t ws_bytes, void* o, int32_t* dev_status, void* stream) {
+  bsa_status s = check_plan(p);
+  if (s != BSA_OK) return s;
+  if (ws == nullptr || ws_bytes < pairing_bytes(p, kmax))
+    return fail(BSA_ERR_WORKSPACE, "paired attention needs the %zu-byte pairing workspace, got %zu",
+                pairing_bytes(p, kmax), ws_bytes);
+  const size_t bh = (size_t)p->g.B * p->g.Hd, pph = pairs_per_head(p->g);
+  const char* w = reinterpret_cast<const char*>(ws) + round256(bsa::pair_scratch_bytes(p->g));
+  const int32_t* sched = reinterpret_cast<const int32_t*>(w);
+  const int32_t* lists = reinterpret_cast<const int32_t*>(w + round256(bh * pph * 4 * sizeof(int32_t)));
+  return run_attention_orig(p, q, k, v, idx, cnt, kmax, o, dev_status, (cudaStream_t)stream,
+                            nullptr, sched, lists);
 }
 
 bsa_status bsa_check_status(bsa_plan_t p, void* stream) {

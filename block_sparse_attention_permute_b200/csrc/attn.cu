@@ -292,10 +292,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int n_tiles = map_count(a.map, g.B * g.Hd) * nbk;
 
   // The two query tiles of this CTA (held in scalars: a runtime-indexed array
-  // would live in local memory).
-  int i0 = -1, i1 = -1, n0 = 0, n1 = 0;
+  // would live in local memory), and how many leading steps they share.
+  int i0 = -1, i1 = -1, n0 = 0, n1 = 0, c_shared = 0;
   long long bh0 = 0, bh1 = 0;
-  {
+  const int32_t* list0;
+  const int32_t* list1;
+  if (a.pair_sched == nullptr) {
     int b, h, i;
     if (2 * (int)blockIdx.x < n_tiles) {
       decode_tile(g, a.map, 2 * blockIdx.x, b, h, i);
@@ -305,9 +307,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       decode_tile(g, a.map, 2 * blockIdx.x + 1, b, h, i);
       i1 = i; bh1 = (long long)b * g.Hd + h; n1 = list_length(g, a, bh1, i);
     }
+    list0 = a.idx + (bh0 * g.nb + (i0 >= 0 && i0 < g.nb ? i0 : 0)) * a.kmax;
+    list1 = a.idx + (bh1 * g.nb + (i1 >= 0 && i1 < g.nb ? i1 : 0)) * a.kmax;
+  } else {
+    // Paired schedule: CTA e covers the text pairs of every head first, then
+    // the video pairs; entry (h, t) names the two tiles and the shared count.
+    const int n_heads = map_count(a.map, g.B * g.Hd);
+    const int vpairs = a.pairs_per_head - a.text_pairs;
+    int e = blockIdx.x, m, t;
+    if (e < n_heads * a.text_pairs) {
+      m = e / a.text_pairs;
+      t = e % a.text_pairs;
+    } else {
+      e -= n_heads * a.text_pairs;
+      m = e / vpairs;
+      t = a.text_pairs + e % vpairs;
+    }
+    const long long bh = map_bh(a.map, m);
+    const long long ent = bh * a.pairs_per_head + t;
+    const int4 se = __ldg(reinterpret_cast<const int4*>(a.pair_sched) + ent);
+    bh0 = bh1 = bh;
+    i0 = se.x;
+    i1 = se.y;
+    if (i0 >= 0) n0 = list_length(g, a, bh, i0);
+    if (i1 >= 0) n1 = list_length(g, a, bh, i1);
+    c_shared = min(se.z, min(n0, n1));
+    list0 = a.pair_lists + (ent * 2 + 0) * a.kmax;
+    list1 = a.pair_lists + (ent * 2 + 1) * a.kmax;
   }
-  const int32_t* list0 = a.idx + (bh0 * g.nb + (i0 >= 0 && i0 < g.nb ? i0 : 0)) * a.kmax;
-  const int32_t* list1 = a.idx + (bh1 * g.nb + (i1 >= 0 && i1 < g.nb ? i1 : 0)) * a.kmax;
   // Key block of step s of tile x; -1 for an out-of-range list entry.
   auto block_at = [&](int x, int s) -> int {
     const int i = x ? i1 : i0;
@@ -347,6 +374,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int pos = 0;
       bool bad = false;
       for_each_event(n0, n1, [&](int kind, int x, int s) -> bool {
+        // tile 1's first c_shared steps use the K / V tiles tile 0 fetched
+        if (x == 1 && s < c_shared) return true;
         int j = block_at(x, s);
         if (j < 0) { bad = true; j = 0; }   // load some tile; the softmax masks the step
         const int slot = pos % L::kStages;
@@ -374,11 +403,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if ((x ? n1 : n0) > 0 && !mbar_wait(bar(L::kBarQ + x), 0, abort)) ok = false;
       tc_fence_after();
       int pos = 0;
+      int shared_slot[2] = {0, 0};   // ring slot of tile 0's K (S) and V (PV) of a shared step
       if (ok) {
         for_each_event(n0, n1, [&](int kind, int x, int s) -> bool {
-          const int slot = pos % L::kStages;
-          if (!mbar_wait(bar(L::kBarFull + slot), (pos / L::kStages) & 1, abort)) return false;
-          tc_fence_after();
+          // a shared step: tile 0 (issued first) waits for the tile and keeps
+          // it; tile 1 reuses it and releases it
+          const bool shared = s < c_shared;
+          int slot;
+          if (shared && x == 1) {
+            slot = kind == 0 ? shared_slot[0] : shared_slot[1];
+          } else {
+            slot = pos % L::kStages;
+            if (!mbar_wait(bar(L::kBarFull + slot), (pos / L::kStages) & 1, abort)) return false;
+            tc_fence_after();
+            ++pos;
+            if (shared) {
+              if (kind == 0) shared_slot[0] = slot;
+              else shared_slot[1] = slot;
+            }
+          }
           const uint32_t src = sRing + slot * kTileBytes;
           const uint32_t tS = tmem + 128u * x;
           if (kind == 0) {
@@ -400,8 +443,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                           (s > 0 || kk > 0) ? 1u : 0u);
             if (s == (x ? n1 : n0) - 1) tc_commit(bar(L::kBarO + x));
           }
-          tc_commit(bar(L::kBarEmpty + slot));
-          ++pos;
+          if (!(shared && x == 0)) tc_commit(bar(L::kBarEmpty + slot));
           return true;
         });
       }
@@ -597,7 +639,9 @@ cudaError_t launch_attn_tc_orig(const Geo& g, const AttnArgs& a, const TileMaps&
                                 cudaStream_t st) {
   const int tiles = map_count(a.map, g.Hd) * (g.nb + g.nb_text);
   if (tiles == 0 || g.B != 1) return g.B != 1 ? cudaErrorInvalidValue : cudaSuccess;
-  const int ctas = (tiles + 1) / 2;
+  // paired schedule: one CTA per entry (a head with an odd tile count has a
+  // single-tile entry)
+  const int ctas = a.pair_sched ? map_count(a.map, g.Hd) * a.pairs_per_head : (tiles + 1) / 2;
   return g.D == 128 ? launch_tc_t<128, true>(g, a, maps, ctas, st)
                     : launch_tc_t<64, true>(g, a, maps, ctas, st);
 }

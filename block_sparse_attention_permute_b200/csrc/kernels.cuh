@@ -83,6 +83,30 @@ struct AttnArgs {
   float scale;            // 1/sqrt(D)
   float scale_log2;       // log2(e)/sqrt(D)
   HeadMap map;
+  // Paired schedule (original-layout path, one batch element per launch), or
+  // null for the plain order (tiles 2x and 2x+1).  Entry (h, t) of a head,
+  // t < text_pairs for its text tiles, then its video pairs:
+  //   pair_sched[(h * pairs_per_head + t) * 4 + {0,1,2}] = {i0, i1 (-1 = none), c}
+  //   pair_lists[((h * pairs_per_head + t) * 2 + x) * kmax + s] = block of step s
+  // The first c steps of both tiles visit the same key blocks (their K and V
+  // tiles are fetched once); video tiles read their lists from pair_lists.
+  const int32_t* pair_sched;
+  const int32_t* pair_lists;
+  int pairs_per_head, text_pairs;
+};
+
+// Pairing of the query tiles of each (b, h) into CTA pairs that share key
+// blocks (pair.cu).
+struct PairArgs {
+  const int32_t* idx;     // [B, Hd, nb, kmax] lists (ascending video blocks, then text)
+  const int32_t* cnt;     // [B, Hd, nb]
+  uint32_t* bits;         // [B * Hd, nb, nbw] scratch: list bit sets
+  uint16_t* cand;         // [B * Hd, nb, 8] scratch: best partners by |L_i & L_j|
+  int32_t* sched;         // [B * Hd, pairs_per_head, 4] out
+  int32_t* lists;         // [B * Hd, pairs_per_head, 2, kmax] out
+  int kmax;
+  int pairs_per_head, text_pairs;
+  HeadMap map;            // pairs of (b, h) to pair up (n = 0: all)
 };
 
 // TMA tensor maps of one attention launch: q/k/v cover the blocked tensors
@@ -101,6 +125,9 @@ cudaError_t launch_sics_schemes(const SchemeArgs& a, bool is_bf16, cudaStream_t 
 size_t select_smem_bytes(int nb, int D);
 cudaError_t launch_select(const Geo& g, const SelectArgs& a, cudaStream_t st);
 cudaError_t launch_intra_select(const Geo& g, const IntraArgs& a, cudaStream_t st);
+// pair.cu
+size_t pair_scratch_bytes(const Geo& g);
+cudaError_t launch_pairing(const Geo& g, const PairArgs& a, cudaStream_t st);
 // attn.cu
 size_t attn_tc_smem_bytes(int D);
 cudaError_t launch_attn_simt(const Geo& g, bool is_bf16, const AttnArgs& a, cudaStream_t st);

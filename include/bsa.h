@@ -451,6 +451,35 @@ bsa_status bsa_forward_grouped(const bsa_plan_t* plans, int n_plans,
                                void* ws, size_t ws_bytes, int32_t* dev_status,
                                void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Tile pairing (no counterpart on the pages: a scheduling step of this
+ * implementation).  The tensor-core attention runs two query tiles per CTA.
+ * bsa_pair_tiles matches the video query blocks of every (b, h) in pairs
+ * whose lists overlap most and writes, into its workspace, a schedule whose
+ * two lists per pair start with the shared blocks; bsa_attention_paired then
+ * fetches each shared K and V tile once for both tiles.  bsa_forward does
+ * both on tensor-core plans.  Lists must be as bsa_select writes them
+ * (ascending video blocks, then every text block).  The result equals
+ * bsa_attention_orig up to the rounding of the reordered sums. */
+
+/* bsa_pair_workspace_size — bytes of the pairing workspace (0 off the
+ * tensor-core path). */
+bsa_status bsa_pair_workspace_size(bsa_plan_t plan, int kmax, size_t* bytes);
+
+/* bsa_pair_tiles — pairs the query tiles of idx / cnt ([B, Hd, nb, kmax],
+ * [B, Hd, nb]) into `ws` (256-byte aligned, >= bsa_pair_workspace_size). */
+bsa_status bsa_pair_tiles(bsa_plan_t plan, const int32_t* idx,
+                          const int32_t* cnt, int kmax, void* ws,
+                          size_t ws_bytes, void* stream);
+
+/* bsa_attention_paired — bsa_attention_orig on the schedule bsa_pair_tiles
+ * wrote into ws from the same idx / cnt. */
+bsa_status bsa_attention_paired(bsa_plan_t plan, const void* q, const void* k,
+                                const void* v, const int32_t* idx,
+                                const int32_t* cnt, int kmax, const void* ws,
+                                size_t ws_bytes, void* o, int32_t* dev_status,
+                                void* stream);
+
 /* bsa_check_status — synchronise `stream`, read and clear the plan-owned
  * status word; returns BSA_OK or the recorded error. */
 bsa_status bsa_check_status(bsa_plan_t plan, void* stream);

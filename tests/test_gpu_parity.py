@@ -140,6 +140,35 @@ def test_attention_on_original_layout(name, dev):
     assert torch.equal(out, blocked)
 
 
+PAIRED = [n for n in SMALL if SMALL[n].dtype == "bf16" and SMALL[n].bs == 128] + ["odd_text"]
+SMALL_EXTRA = {"odd_text": custom_workload("odd_text", 2, 5, 9, 20, 1, 8, 16, 2, 128, 300, "bf16",
+                                           0, 0.4)}
+
+
+@pytest.mark.parametrize("name", PAIRED)
+def test_paired_attention(name, dev):
+    """Tile pairing (shared key blocks first) changes only the summation order:
+    the output matches the oracle over the same lists, and bsa_forward (which
+    pairs) equals pair_tiles + attention_paired bit for bit."""
+    w = SMALL[name] if name in SMALL else SMALL_EXTRA[name]
+    g = geometry(w)
+    (q, k, v), (qd, kd, vd) = _inputs(w, dev)
+    plan = bsa.plan_for(w, dev)
+    qc, kc = plan.centroids(qd, kd)
+    idx, cnt = plan.select_centroids(qc, kc, w.mode, w.params)
+    ws = plan.pair_tiles(idx, cnt)
+    out = plan.attention_paired(qd, kd, vd, idx, cnt, ws)
+    unpaired = plan.attention_orig(qd, kd, vd, idx, cnt)
+    fwd = plan.forward(qd, kd, vd, w.mode, w.params)
+    plan.check_status()
+    ref = orc.attention(g, to_np(q), to_np(k), to_np(v), idx.cpu().numpy(), cnt.cpu().numpy())
+    check_output(to_np(out), ref, w.dtype, f"{name} paired")
+    check_output(to_np(unpaired), ref, w.dtype, f"{name} unpaired")
+    assert torch.equal(fwd, out)
+    print(f"{name}: nb={g.nb} nb_text={g.nb_text} max |paired - unpaired| = "
+          f"{float((out.float() - unpaired.float()).abs().max()):.2e}")
+
+
 def test_attention_on_original_layout_needs_tensor_core_plan(dev):
     w = SMALL["simt_bf16_bs32"]
     (_, _, _), (qd, kd, vd) = _inputs(w, dev)
