@@ -5,7 +5,8 @@
 // differ per query block, so two arbitrary tiles rarely need the same K/V
 // tiles; but the lists of query blocks with similar summaries overlap
 // strongly.  Here each (b, h)'s video query blocks are matched in pairs with
-// large overlap |L_i & L_j|: every block keeps its kCand best partners, and
+// large overlap |L_i & L_j|: every block keeps its kCand best partners among
+// its neighbours in block order (a window reaching the next frame), and
 // in a few "mutual best partner" rounds a block and its best unmatched
 // candidate are matched when each is the other's; the rest are paired in
 // index order.  Each pair's two lists are reordered so that the shared
@@ -52,51 +53,63 @@ __global__ void __launch_bounds__(256) pair_bits_kernel(Geo g, PairArgs a) {
 }
 
 // Candidate partners of every query block: its kCand largest overlaps
-// |L_i & L_j| (j != i; equal overlaps to the smaller j), one warp per
-// (bh, i), 16 rows per CTA; lane l holds the overlaps with j = l + 32 t in
-// registers.  The head's bit sets are staged in shared memory with an odd
-// row stride (conflict-free column reads) when they fit, else read from L2.
+// |L_i & L_j| over the blocks j within `win` of i in block order (j != i;
+// equal overlaps to the smaller j).  The window covers the neighbours of a
+// block in x, y and t (a t-neighbour is nbx * nby blocks away); blocks that
+// far apart rarely share more keys than the near ones, and searching all nb
+// blocks cost nb^2 popcount rows per head.  One warp per (bh, i), kCandRows
+// rows per CTA; lane l holds the overlaps with j = i - win + l + 32 t in
+// registers.  The bit sets of rows [i0 - win, i0 + kCandRows + win) are
+// staged in shared memory with an odd row stride (conflict-free column reads).
 constexpr int kCandRows = 16;
+constexpr int kWinT = 8;   // at most 8 * 32 candidates per block: win <= 127
 
-template <bool SMEM>
-__global__ void __launch_bounds__(kCandRows * 32) pair_cand_kernel(Geo g, PairArgs a) {
+int pair_window_lanes(const Geo& g) {
+  const long long w0 = (long long)g.nbx * g.nby + g.nbx + 1;
+  const long long t = (2 * w0 + 1 + 31) / 32;
+  return (int)(t < kWinT ? t : kWinT);
+}
+size_t pair_cand_smem(const Geo& g) {
+  const int win = (32 * pair_window_lanes(g) - 1) / 2;
+  const int nbw = (g.nb + 31) / 32;
+  return (size_t)(kCandRows + 2 * win) * (nbw | 1) * sizeof(uint32_t);
+}
+
+__global__ void __launch_bounds__(kCandRows * 32) pair_cand_kernel(Geo g, PairArgs a, int n_t) {
   extern __shared__ uint32_t s_bits_all[];
   const int bh = map_bh(a.map, blockIdx.x);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = blockIdx.y * kCandRows + warp;
-  const int nbw = (g.nb + 31) / 32;
-  const int stride = SMEM ? (nbw | 1) : nbw;
-  const uint32_t* gbits = a.bits + (long long)bh * g.nb * nbw;
-  const uint32_t* bits = gbits;
-  if (SMEM) {
-    for (int e = threadIdx.x; e < g.nb * nbw; e += blockDim.x)
-      s_bits_all[(e / nbw) * stride + e % nbw] = gbits[e];
-    __syncthreads();
-    bits = s_bits_all;
-  }
-  __shared__ uint32_t s_row[kCandRows][kMaxWords];
-  if (i >= g.nb) return;
-  for (int w = lane; w < nbw; w += 32) s_row[warp][w] = gbits[(long long)i * nbw + w];
-  __syncwarp();
-  int ov[kMaxWords];   // -1: no such j, or already picked
+  const int nb = g.nb, nbw = (nb + 31) / 32, stride = nbw | 1;
+  const int win = (32 * n_t - 1) / 2;
+  const int i0 = blockIdx.y * kCandRows;
+  const int lo = max(0, i0 - win), hi = min(nb, i0 + kCandRows + win);
+  const uint32_t* gbits = a.bits + (long long)bh * nb * nbw;
+  for (int e = threadIdx.x; e < (hi - lo) * nbw; e += blockDim.x)
+    s_bits_all[(e / nbw) * stride + e % nbw] = gbits[(long long)lo * nbw + e];
+  __syncthreads();
+  const int i = i0 + warp;
+  if (i >= nb) return;
+  const uint32_t* row_i = s_bits_all + (i - lo) * stride;
+  const int jbase = i - win;   // j of (lane 0, t = 0)
+  int ov[kWinT];   // -1: no such j, or already picked
 #pragma unroll
-  for (int t = 0; t < kMaxWords; ++t) {
-    const int j = lane + 32 * t;
+  for (int t = 0; t < kWinT; ++t) {
+    const int j = jbase + lane + 32 * t;
     int c = -1;
-    if (j < g.nb && j != i) {
+    if (t < n_t && lane + 32 * t <= 2 * win && j >= 0 && j < nb && j != i) {
       c = 0;
-      const uint32_t* bj = bits + (long long)j * stride;
-      for (int w = 0; w < nbw; ++w) c += __popc(s_row[warp][w] & bj[w]);
+      const uint32_t* row_j = s_bits_all + (j - lo) * stride;
+      for (int w = 0; w < nbw; ++w) c += __popc(row_i[w] & row_j[w]);
     }
     ov[t] = c;
   }
-  uint16_t* out = a.cand + ((long long)bh * g.nb + i) * kCand;
+  uint16_t* out = a.cand + ((long long)bh * nb + i) * kCand;
   for (int k = 0; k < kCand; ++k) {
     int bv = -1, bt = -1;
 #pragma unroll
-    for (int t = 0; t < kMaxWords; ++t)
+    for (int t = 0; t < kWinT; ++t)
       if (ov[t] > bv) { bv = ov[t]; bt = t; }
-    int bj = bt >= 0 ? lane + 32 * bt : -1;
+    int bj = bt >= 0 ? jbase + lane + 32 * bt : -1;
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) {
       const int v2 = __shfl_xor_sync(0xffffffffu, bv, o);
@@ -104,10 +117,11 @@ __global__ void __launch_bounds__(kCandRows * 32) pair_cand_kernel(Geo g, PairAr
       if (v2 > bv || (v2 == bv && j2 >= 0 && (bj < 0 || j2 < bj))) { bv = v2; bj = j2; }
     }
     if (lane == 0) out[k] = bj < 0 ? (uint16_t)0xffffu : (uint16_t)bj;
-    if (bj >= 0 && (bj & 31) == lane) {   // remove the pick from its lane
+    if (bj >= 0 && ((bj - jbase) & 31) == lane) {   // remove the pick from its lane
+      const int tp = (bj - jbase) >> 5;
 #pragma unroll
-      for (int t = 0; t < kMaxWords; ++t)
-        if (t == (bj >> 5)) ov[t] = -1;
+      for (int t = 0; t < kWinT; ++t)
+        if (t == tp) ov[t] = -1;
     }
   }
 }
@@ -296,17 +310,11 @@ cudaError_t launch_pairing(const Geo& g, const PairArgs& a, cudaStream_t st) {
   pair_bits_kernel<<<dim3(n_bh, (g.nb + 7) / 8), 256, 0, st>>>(g, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int nbw = (g.nb + 31) / 32;
-  const size_t cand_smem = (size_t)g.nb * (nbw | 1) * sizeof(uint32_t);
+  const size_t cand_smem = pair_cand_smem(g);   // <= 270 rows x 49 words
   const dim3 cgrid(n_bh, (g.nb + kCandRows - 1) / kCandRows);
-  if (cand_smem <= 200 * 1024) {
-    e = cudaFuncSetAttribute(pair_cand_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)cand_smem);
-    if (e != cudaSuccess) return e;
-    pair_cand_kernel<true><<<cgrid, kCandRows * 32, cand_smem, st>>>(g, a);
-  } else {
-    pair_cand_kernel<false><<<cgrid, kCandRows * 32, 0, st>>>(g, a);
-  }
+  e = cudaFuncSetAttribute(pair_cand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cand_smem);
+  if (e != cudaSuccess) return e;
+  pair_cand_kernel<<<cgrid, kCandRows * 32, cand_smem, st>>>(g, a, pair_window_lanes(g));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const size_t smem = 5 * (size_t)g.nb * sizeof(int);
   if (smem > 48 * 1024) {

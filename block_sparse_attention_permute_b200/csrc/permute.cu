@@ -213,6 +213,63 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(Geo g, GatherArg
   gather_block<T, D, MODE, EXTRAS>(g, src, dst, cent, sics, box, blockIdx.x, bh % g.Hd, bh / g.Hd);
 }
 
+// Centroids of the video blocks from the original layout, bf16 plans with
+// 128-token blocks (the summarizer pass of bsa_forward).  One CTA of 128
+// threads per (tensor, block j, group of heads); thread (head, v) owns the
+// 16-byte column v of one head and streams it through the block's 128 slots,
+// so a warp reads whole runs of adjacent heads of one token and no partial
+// sums cross threads.  The sums are formed in the order of gather_block's
+// kPool path (row group r = s mod R holds s = r, r + R, ...; the groups are
+// then added in ascending r), so the centroids are bit-identical to the
+// blocked-layout pool.
+constexpr int kColThreads = 128;
+
+template <int D>
+__global__ void __launch_bounds__(kColThreads) pool_cols_kernel(Geo g, GatherArgs a) {
+  using T = __nv_bfloat16;
+  constexpr int E = 8;                      // bf16 elements per 16-byte vector
+  constexpr int V = D / E;                  // vectors per row
+  constexpr int R = kGatherThreads / V;     // row groups, as in gather_block
+  constexpr int M = 128 / R;                // rows per group
+  constexpr int HG = kColThreads / V;       // heads per CTA
+  __shared__ int s_tok[128];
+  const int j = blockIdx.x, t = blockIdx.z;
+  const int p = blockIdx.y * HG + (int)threadIdx.x / V, vec = (int)threadIdx.x % V;
+  const void* src_ptr = t == 0 ? a.src[0] : t == 1 ? a.src[1] : a.src[2];
+  float* cent = t == 0 ? a.cent[0] : t == 1 ? a.cent[1] : a.cent[2];
+  s_tok[threadIdx.x] = (int)slot_token(g, j, threadIdx.x);
+  __syncthreads();
+  if (p >= map_count(a.map, g.B * g.Hd) || cent == nullptr) return;
+  const int bh = map_bh(a.map, p), b = bh / g.Hd, h = bh % g.Hd;
+  const uint4* src = reinterpret_cast<const uint4*>(src_ptr) + ((long long)b * g.n_tot * g.Hd + h) * V + vec;
+  const long long tok_stride = (long long)g.Hd * V;   // uint4 per token
+  float total[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) total[e] = 0.f;
+#pragma unroll 2
+  for (int r = 0; r < R; ++r) {
+    uint4 x[M];
+    int tok[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      tok[m] = s_tok[r + R * m];
+      x[m] = tok[m] >= 0 ? __ldg(src + tok[m] * tok_stride) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float part[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) part[e] = 0.f;
+#pragma unroll
+    for (int m = 0; m < M; ++m)
+      if (tok[m] >= 0) accumulate_vec<T>(part, x[m]);
+#pragma unroll
+    for (int e = 0; e < E; ++e) total[e] += part[e];
+  }
+  const float n = (float)block_valid_count(g, j);
+  float4* out = reinterpret_cast<float4*>(cent + ((long long)bh * g.nb + j) * D + vec * E);
+  out[0] = make_float4(total[0] / n, total[1] / n, total[2] / n, total[3] / n);
+  out[1] = make_float4(total[4] / n, total[5] / n, total[6] / n, total[7] / n);
+}
+
 // Aggregation evaluation (SPADE §3.2): SICS of every block of every candidate
 // blocking scheme, read from the original layout.  One warp per (b, h,
 // candidate, block): the online form of Eq. (5), a running sum of unit rows
@@ -230,18 +287,6 @@ constexpr int kSicsWarps = 4;
 constexpr int kSicsStages = 4;
 constexpr int kSicsChunks = 4;
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kSicsWarps * 32, 4) sics_schemes_kernel(SchemeArgs s, int per_bh,
@@ -406,6 +451,17 @@ cudaError_t launch_unpermute(const Geo& g, bool is_bf16, const GatherArgs& a, cu
 // summarizer pass of the fused forward, which never materialises the blocked
 // tensors).
 cudaError_t launch_pool_orig(const Geo& g, bool is_bf16, const GatherArgs& a, cudaStream_t st) {
+  bool extras = false;
+  for (int t = 0; t < a.ntensors; ++t) extras = extras || a.sics[t] != nullptr || a.box[t] != nullptr;
+  if (is_bf16 && g.bs == 128 && !extras && (g.D == 128 || g.D == 64)) {
+    const int pairs = map_count(a.map, g.B * g.Hd);
+    const int hg = kColThreads / (g.D / 8);
+    const dim3 grid(g.nb, (pairs + hg - 1) / hg, a.ntensors);
+    if (g.nb == 0 || pairs == 0) return cudaSuccess;
+    if (g.D == 128) pool_cols_kernel<128><<<grid, kColThreads, 0, st>>>(g, a);
+    else pool_cols_kernel<64><<<grid, kColThreads, 0, st>>>(g, a);
+    return cudaGetLastError();
+  }
   return is_bf16 ? launch_gather_t<__nv_bfloat16, kPoolOrig>(g, a, g.nb, st)
                  : launch_gather_t<float, kPoolOrig>(g, a, g.nb, st);
 }

@@ -24,11 +24,14 @@ namespace bsa {
 
 constexpr int kSelRows = 16;      // query-block rows per CTA
 constexpr int kSelKeys = 256;     // key blocks per score chunk
-constexpr int kSelDChunk = 32;    // head-dim slice of a key chunk held in shared memory
+constexpr int kSelDChunk = 16;    // head-dim slice of a key chunk held in shared memory
+constexpr int kSelKS = kSelDChunk + 4;   // padded chunk row: conflict-free float4 reads
 constexpr int kSelThreads = 256;  // 8 warps
 
+// query summaries, two key-chunk buffers (the next chunk lands while the
+// current one is used), the score rows
 size_t select_smem_bytes(int nb, int D) {
-  return sizeof(float) * ((size_t)kSelRows * D + (size_t)kSelKeys * (kSelDChunk + 4) +
+  return sizeof(float) * ((size_t)kSelRows * D + 2 * (size_t)kSelKeys * kSelKS +
                           (size_t)kSelRows * nb);
 }
 
@@ -77,22 +80,78 @@ __device__ int count_at_least(const float* row, int nb, uint32_t cand, int lane)
   return c;
 }
 
-// Lanes hold the order keys of their scores (j = lane + 32 e) in registers,
-// so the 32-step threshold search does not re-read shared memory.
+// Lanes hold the order keys of their scores (j = lane + 32 e) in registers
+// (and, for Top-P, their weights), so the 32-step threshold search neither
+// re-reads shared memory nor recomputes a weight; the register count per
+// lane is the smallest of 16, 32, 48 that covers the row.
 constexpr int kKeysPerLane = 48;   // register-resident search for nb <= 1536
 
-// Largest T with #{j : key_j >= T} >= k (the k-th largest key), bit by bit.
-__device__ __forceinline__ uint32_t kth_largest_key(const uint32_t (&kr)[kKeysPerLane], int k) {
+// Threshold of the Top-K / Top-P rule over one row with the keys (and, for
+// Top-P, the weights) in registers.  Every sum runs over j = lane + 32 e in
+// ascending e, then across the warp, as in mass_at_least, so the fp64 masses
+// are those of the shared-memory loops below.
+template <int KPL, bool TOPP, class Wt>
+__device__ __forceinline__ void rule_threshold_regs(const float* row, int nb, int k, double target,
+                                                    Wt wt, int lane, uint32_t* T_out, int* need_out) {
+  // order_key of any float is nonzero and every candidate threshold is
+  // nonzero, so the 0 used for missing entries never counts
+  uint32_t kr[KPL];
+  float wf[TOPP ? KPL : 1];   // weight of each score (0 for missing entries)
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    const int j = lane + 32 * e;
+    const float sv = j < nb ? row[j] : 0.f;
+    kr[e] = j < nb ? order_key(sv) : 0u;
+    if (TOPP) wf[e] = j < nb ? (float)wt(sv) : 0.f;
+  }
   uint32_t T = 0;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = T | (1u << bit);
+  int need = 0;
+  if (!TOPP) {
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      int c = 0;
+#pragma unroll
+      for (int e = 0; e < KPL; ++e) c += kr[e] >= cand ? 1 : 0;
+      c = __reduce_add_sync(0xffffffffu, c);
+      if (c >= k) T = cand;
+    }
     int c = 0;
 #pragma unroll
-    for (int e = 0; e < kKeysPerLane; ++e) c += kr[e] >= cand ? 1 : 0;   // pad keys are 0
-    c = __reduce_add_sync(0xffffffffu, c);
-    if (c >= k) T = cand;
+    for (int e = 0; e < KPL; ++e) c += kr[e] > T ? 1 : 0;
+    need = k - __reduce_add_sync(0xffffffffu, c);
+  } else {
+    // mass of the keys >= cand; a weight is a float widened exactly to fp64
+    auto mass = [&](uint32_t cand) -> double {
+      double acc = 0.0;
+#pragma unroll
+      for (int e = 0; e < KPL; ++e)
+        if (kr[e] >= cand) acc += (double)wf[TOPP ? e : 0];   // cand >= 1: missing entries never count
+      return warp_sum_uniform(acc);
+    };
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      if (mass(cand) >= target) T = cand;
+    }
+    double acc = (T == 0xffffffffu) ? 0.0 : mass(T + 1);
+    int n_eq = 0;
+    float s_eq = 0.f;
+#pragma unroll
+    for (int e = 0; e < KPL; ++e)
+      if (kr[e] == T && lane + 32 * e < nb) { ++n_eq; s_eq = row[lane + 32 * e]; }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      n_eq += __shfl_xor_sync(0xffffffffu, n_eq, off);
+      s_eq = fmaxf(s_eq, __shfl_xor_sync(0xffffffffu, s_eq, off));
+    }
+    const double e_eq = wt(s_eq);
+    while (acc < target && need < n_eq) {
+      acc += e_eq;
+      ++need;
+    }
+    if (need == 0) need = 1;
   }
-  return T;
+  *T_out = T;
+  *need_out = need;
 }
 
 // Threshold of the Top-K / Top-P rule over one row of nb scores: every entry
@@ -111,30 +170,28 @@ __device__ __forceinline__ void rule_threshold(const float* row, int nb, int mod
     mode = 0;
     param = 1.0;
   }
+  // Registers: Top-K keeps up to 48 keys per lane, Top-P up to 32 keys and
+  // their weights; longer rows use the shared-memory loops.
+  if (mode == 0 && nb <= 32 * kKeysPerLane) {
+    const int k = (int)param;
+    if (nb <= 32 * 16) rule_threshold_regs<16, false>(row, nb, k, target, wt, lane, T_out, need_out);
+    else if (nb <= 32 * 32) rule_threshold_regs<32, false>(row, nb, k, target, wt, lane, T_out, need_out);
+    else rule_threshold_regs<kKeysPerLane, false>(row, nb, k, target, wt, lane, T_out, need_out);
+    return;
+  }
+  if (mode != 0 && nb <= 32 * 32) {
+    if (nb <= 32 * 16) rule_threshold_regs<16, true>(row, nb, 0, target, wt, lane, T_out, need_out);
+    else rule_threshold_regs<32, true>(row, nb, 0, target, wt, lane, T_out, need_out);
+    return;
+  }
   if (mode == 0) {
     const int k = (int)param;
-    if (nb <= 32 * kKeysPerLane) {
-      // order_key of any float is nonzero and every candidate threshold is
-      // nonzero, so the 0 used for missing entries never counts
-      uint32_t kr[kKeysPerLane];
-#pragma unroll
-      for (int e = 0; e < kKeysPerLane; ++e) {
-        const int j = lane + 32 * e;
-        kr[e] = j < nb ? order_key(row[j]) : 0u;
-      }
-      T = kth_largest_key(kr, k);
-      int c = 0;
-#pragma unroll
-      for (int e = 0; e < kKeysPerLane; ++e) c += kr[e] > T ? 1 : 0;
-      need = k - __reduce_add_sync(0xffffffffu, c);
-    } else {
-      for (int bit = 31; bit >= 0; --bit) {
-        const uint32_t cand = T | (1u << bit);
-        if (count_at_least(row, nb, cand, lane) >= k) T = cand;
-      }
-      const int n_gt = (T == 0xffffffffu) ? 0 : count_at_least(row, nb, T + 1, lane);
-      need = k - n_gt;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      if (count_at_least(row, nb, cand, lane) >= k) T = cand;
     }
+    const int n_gt = (T == 0xffffffffu) ? 0 : count_at_least(row, nb, T + 1, lane);
+    need = k - n_gt;
   } else {
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = T | (1u << bit);
@@ -178,8 +235,8 @@ template <int D, int EST>
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(Geo g, SelectArgs a) {
   extern __shared__ __align__(16) float sm[];
   float* qs = sm;                                   // [kSelRows][D]
-  float* ks = qs + kSelRows * D;                    // [kSelKeys][kSelDChunk+4]
-  float* sc = ks + kSelKeys * (kSelDChunk + 4);     // [kSelRows][nb]
+  float* ks = qs + kSelRows * D;                    // [2][kSelKeys][kSelKS]
+  float* sc = ks + 2 * kSelKeys * kSelKS;           // [kSelRows][nb]
   const int nb = g.nb;
   const int bhi = map_bh(a.map, (int)blockIdx.z * g.Hd + (int)blockIdx.y);
   const int h = bhi % g.Hd, b = bhi / g.Hd;
@@ -189,8 +246,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(Geo g, SelectArg
 
   // ---- phase 1: scores of kSelRows query blocks against all key blocks ----
   // Thread (ty, tx) accumulates rows 8ty..8ty+7 against keys tx and tx+128 of
-  // each 256-key chunk; the chunk's keys pass through shared memory 32
-  // dimensions at a time.  Each dot product is one fma chain over d in
+  // each 256-key chunk; the chunk's keys pass through shared memory 16
+  // dimensions at a time (double-buffered).  Each dot product is one fma chain over d in
   // ascending order, the same as a plain sequential loop.
   if (EST == kEstDsa) {
     // DSA: the query summary is the box centre c = (max + min) / 2, stored as
@@ -214,51 +271,71 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(Geo g, SelectArg
     }
   }
   const int ty = tid / 128, tx = tid % 128;
-  constexpr int KS = kSelDChunk + 4;               // padded row: conflict-free float4 reads
-  for (int j0 = 0; j0 < nb; j0 += kSelKeys) {
-    float acc[8][2];
+  // The key chunks (kSelKeys key blocks x kSelDChunk dimensions) are visited
+  // j0-major; chunk c + 1 is copied with cp.async into the other buffer while
+  // chunk c is used.  Rows past nb are zero-filled.
+  constexpr int kDChunks = D / kSelDChunk;
+  const int n_chunks = ((nb + kSelKeys - 1) / kSelKeys) * kDChunks;
+  const float* kc_bh = a.kc + bh * nb * D;
+  auto issue_chunk = [&](int c) {
+    const int j0 = (c / kDChunks) * kSelKeys, d0 = (c % kDChunks) * kSelDChunk;
+    float* buf = ks + (c & 1) * kSelKeys * kSelKS;
+    for (int e = tid; e < kSelKeys * (kSelDChunk / 4); e += kSelThreads) {
+      const int jj = e / (kSelDChunk / 4), d4 = e % (kSelDChunk / 4);
+      const bool ok = j0 + jj < nb;
+      cp_async16(smem_addr(buf + jj * kSelKS + 4 * d4),
+                 ok ? kc_bh + (long long)(j0 + jj) * D + d0 + 4 * d4 : kc_bh, ok ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
+  issue_chunk(0);
+  float acc[8][2];
+  for (int c = 0; c < n_chunks; ++c) {
+    const int j0 = (c / kDChunks) * kSelKeys, d0 = (c % kDChunks) * kSelDChunk;
+    if (d0 == 0) {
 #pragma unroll
-    for (int r = 0; r < 8; ++r) acc[r][0] = acc[r][1] = 0.f;
-    for (int d0 = 0; d0 < D; d0 += kSelDChunk) {
-      __syncthreads();
-      for (int e = tid; e < kSelKeys * (kSelDChunk / 4); e += kSelThreads) {
-        const int jj = e / (kSelDChunk / 4), d4 = e % (kSelDChunk / 4);
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (j0 + jj < nb)
-          v = *reinterpret_cast<const float4*>(a.kc + (bh * nb + j0 + jj) * D + d0 + 4 * d4);
-        *reinterpret_cast<float4*>(ks + jj * KS + 4 * d4) = v;
-      }
-      __syncthreads();
+      for (int r = 0; r < 8; ++r) acc[r][0] = acc[r][1] = 0.f;
+    }
+    if (c + 1 < n_chunks) {
+      issue_chunk(c + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();   // chunk c (and, at c = 0, the query summaries) visible
+    const float* kb = ks + (c & 1) * kSelKeys * kSelKS;
 #pragma unroll
-      for (int d4 = 0; d4 < kSelDChunk / 4; ++d4) {
-        const float4 k0 = *reinterpret_cast<const float4*>(ks + tx * KS + 4 * d4);
-        const float4 k1 = *reinterpret_cast<const float4*>(ks + (tx + 128) * KS + 4 * d4);
+    for (int d4 = 0; d4 < kSelDChunk / 4; ++d4) {
+      const float4 k0 = *reinterpret_cast<const float4*>(kb + tx * kSelKS + 4 * d4);
+      const float4 k1 = *reinterpret_cast<const float4*>(kb + (tx + 128) * kSelKS + 4 * d4);
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          const float4 qv = *reinterpret_cast<const float4*>(qs + (8 * ty + r) * D + d0 + 4 * d4);
-          if (EST == kEstDsa2) {
-            acc[r][0] += box_max_product(qv.x, qv.y, k0.x, k0.y);
-            acc[r][0] += box_max_product(qv.z, qv.w, k0.z, k0.w);
-            acc[r][1] += box_max_product(qv.x, qv.y, k1.x, k1.y);
-            acc[r][1] += box_max_product(qv.z, qv.w, k1.z, k1.w);
-            continue;
-          }
-          acc[r][0] = fmaf(qv.x, k0.x, acc[r][0]);
-          acc[r][0] = fmaf(qv.y, k0.y, acc[r][0]);
-          acc[r][0] = fmaf(qv.z, k0.z, acc[r][0]);
-          acc[r][0] = fmaf(qv.w, k0.w, acc[r][0]);
-          acc[r][1] = fmaf(qv.x, k1.x, acc[r][1]);
-          acc[r][1] = fmaf(qv.y, k1.y, acc[r][1]);
-          acc[r][1] = fmaf(qv.z, k1.z, acc[r][1]);
-          acc[r][1] = fmaf(qv.w, k1.w, acc[r][1]);
+      for (int r = 0; r < 8; ++r) {
+        const float4 qv = *reinterpret_cast<const float4*>(qs + (8 * ty + r) * D + d0 + 4 * d4);
+        if (EST == kEstDsa2) {
+          acc[r][0] += box_max_product(qv.x, qv.y, k0.x, k0.y);
+          acc[r][0] += box_max_product(qv.z, qv.w, k0.z, k0.w);
+          acc[r][1] += box_max_product(qv.x, qv.y, k1.x, k1.y);
+          acc[r][1] += box_max_product(qv.z, qv.w, k1.z, k1.w);
+          continue;
         }
+        acc[r][0] = fmaf(qv.x, k0.x, acc[r][0]);
+        acc[r][0] = fmaf(qv.y, k0.y, acc[r][0]);
+        acc[r][0] = fmaf(qv.z, k0.z, acc[r][0]);
+        acc[r][0] = fmaf(qv.w, k0.w, acc[r][0]);
+        acc[r][1] = fmaf(qv.x, k1.x, acc[r][1]);
+        acc[r][1] = fmaf(qv.y, k1.y, acc[r][1]);
+        acc[r][1] = fmaf(qv.z, k1.z, acc[r][1]);
+        acc[r][1] = fmaf(qv.w, k1.w, acc[r][1]);
       }
     }
+    if (d0 + kSelDChunk == D) {
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      if (j0 + tx < nb) sc[(8 * ty + r) * nb + j0 + tx] = acc[r][0] * a.scale + 0.0f;
-      if (j0 + tx + 128 < nb) sc[(8 * ty + r) * nb + j0 + tx + 128] = acc[r][1] * a.scale + 0.0f;
+      for (int r = 0; r < 8; ++r) {
+        if (j0 + tx < nb) sc[(8 * ty + r) * nb + j0 + tx] = acc[r][0] * a.scale + 0.0f;
+        if (j0 + tx + 128 < nb) sc[(8 * ty + r) * nb + j0 + tx + 128] = acc[r][1] * a.scale + 0.0f;
+      }
     }
+    __syncthreads();   // buffer (c & 1) is refilled by the copy issued next iteration
   }
   __syncthreads();
 
