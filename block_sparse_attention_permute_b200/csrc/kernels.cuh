@@ -122,7 +122,7 @@ cudaError_t launch_unpermute(const Geo& g, bool is_bf16, const GatherArgs& a, cu
 cudaError_t launch_pool(const Geo& g, bool is_bf16, const GatherArgs& a, cudaStream_t st);
 cudaError_t launch_sics_schemes(const SchemeArgs& a, bool is_bf16, cudaStream_t st);
 // select.cu
-size_t select_smem_bytes(int nb, int D);
+size_t select_smem_bytes(int nb, int D, int rows = 16);   // rows: query blocks per CTA
 cudaError_t launch_select(const Geo& g, const SelectArgs& a, cudaStream_t st);
 cudaError_t launch_intra_select(const Geo& g, const IntraArgs& a, cudaStream_t st);
 // pair.cu

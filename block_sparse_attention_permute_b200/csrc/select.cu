@@ -22,7 +22,7 @@
 namespace bsa {
 
 
-constexpr int kSelRows = 16;      // query-block rows per CTA
+constexpr int kSelRows = 16;      // query-block rows per CTA (8 for long rows, see launch_select_t)
 constexpr int kSelKeys = 256;     // key blocks per score chunk
 constexpr int kSelDChunk = 16;    // head-dim slice of a key chunk held in shared memory
 constexpr int kSelKS = kSelDChunk + 4;   // padded chunk row: conflict-free float4 reads
@@ -30,9 +30,8 @@ constexpr int kSelThreads = 256;  // 8 warps
 
 // query summaries, two key-chunk buffers (the next chunk lands while the
 // current one is used), the score rows
-size_t select_smem_bytes(int nb, int D) {
-  return sizeof(float) * ((size_t)kSelRows * D + 2 * (size_t)kSelKeys * kSelKS +
-                          (size_t)kSelRows * nb);
+size_t select_smem_bytes(int nb, int D, int rows) {
+  return sizeof(float) * ((size_t)rows * D + 2 * (size_t)kSelKeys * kSelKS + (size_t)rows * nb);
 }
 
 __device__ __forceinline__ uint32_t order_key(float s) {
@@ -107,13 +106,19 @@ __device__ __forceinline__ void rule_threshold_regs(const float* row, int nb, in
   uint32_t T = 0;
   int need = 0;
   if (!TOPP) {
+    // Once exactly k keys reach a candidate, {key >= cand} is the Top-K set
+    // (the same set the full search's threshold, the k-th key, selects) and
+    // the search can stop there.
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = T | (1u << bit);
       int c = 0;
 #pragma unroll
       for (int e = 0; e < KPL; ++e) c += kr[e] >= cand ? 1 : 0;
       c = __reduce_add_sync(0xffffffffu, c);
-      if (c >= k) T = cand;
+      if (c >= k) {
+        T = cand;
+        if (c == k) break;
+      }
     }
     int c = 0;
 #pragma unroll
@@ -231,28 +236,29 @@ __device__ __forceinline__ float box_max_product(float aM, float am, float bM, f
 
 // D = length of the stored summary vectors (head_dim for MEAN, 2 * head_dim
 // for the (max, min) boxes of DSA and DSA2).
-template <int D, int EST>
+template <int D, int EST, int ROWS>
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(Geo g, SelectArgs a) {
+  constexpr int RPT = ROWS / 2;                     // rows per thread in phase 1
   extern __shared__ __align__(16) float sm[];
-  float* qs = sm;                                   // [kSelRows][D]
-  float* ks = qs + kSelRows * D;                    // [2][kSelKeys][kSelKS]
-  float* sc = ks + 2 * kSelKeys * kSelKS;           // [kSelRows][nb]
+  float* qs = sm;                                   // [ROWS][D]
+  float* ks = qs + ROWS * D;                        // [2][kSelKeys][kSelKS]
+  float* sc = ks + 2 * kSelKeys * kSelKS;           // [ROWS][nb]
   const int nb = g.nb;
   const int bhi = map_bh(a.map, (int)blockIdx.z * g.Hd + (int)blockIdx.y);
   const int h = bhi % g.Hd, b = bhi / g.Hd;
   const long long bh = (long long)b * g.Hd + h;
-  const int i0 = blockIdx.x * kSelRows;
+  const int i0 = blockIdx.x * ROWS;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  // ---- phase 1: scores of kSelRows query blocks against all key blocks ----
-  // Thread (ty, tx) accumulates rows 8ty..8ty+7 against keys tx and tx+128 of
+  // ---- phase 1: scores of ROWS query blocks against all key blocks ----
+  // Thread (ty, tx) accumulates rows RPT ty .. RPT ty + RPT - 1 against keys tx and tx+128 of
   // each 256-key chunk; the chunk's keys pass through shared memory 16
   // dimensions at a time (double-buffered).  Each dot product is one fma chain over d in
   // ascending order, the same as a plain sequential loop.
   if (EST == kEstDsa) {
     // DSA: the query summary is the box centre c = (max + min) / 2, stored as
     // (c+, c-) pairs so that c+ kmax + c- kmin = max(c kmax, c kmin)
-    for (int e = tid; e < kSelRows * D / 2; e += kSelThreads) {
+    for (int e = tid; e < ROWS * D / 2; e += kSelThreads) {
       const int r = e / (D / 2), d = e % (D / 2);
       float cp = 0.f, cn = 0.f;
       if (i0 + r < nb) {
@@ -265,7 +271,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(Geo g, SelectArg
       qs[r * D + 2 * d + 1] = cn;
     }
   } else {
-    for (int e = tid; e < kSelRows * D; e += kSelThreads) {
+    for (int e = tid; e < ROWS * D; e += kSelThreads) {
       const int r = e / D, d = e % D;
       qs[e] = (i0 + r < nb) ? a.qc[(bh * nb + i0 + r) * D + d] : 0.f;
     }
@@ -289,12 +295,12 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(Geo g, SelectArg
     cp_async_commit();
   };
   issue_chunk(0);
-  float acc[8][2];
+  float acc[RPT][2];
   for (int c = 0; c < n_chunks; ++c) {
     const int j0 = (c / kDChunks) * kSelKeys, d0 = (c % kDChunks) * kSelDChunk;
     if (d0 == 0) {
 #pragma unroll
-      for (int r = 0; r < 8; ++r) acc[r][0] = acc[r][1] = 0.f;
+      for (int r = 0; r < RPT; ++r) acc[r][0] = acc[r][1] = 0.f;
     }
     if (c + 1 < n_chunks) {
       issue_chunk(c + 1);
@@ -309,8 +315,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(Geo g, SelectArg
       const float4 k0 = *reinterpret_cast<const float4*>(kb + tx * kSelKS + 4 * d4);
       const float4 k1 = *reinterpret_cast<const float4*>(kb + (tx + 128) * kSelKS + 4 * d4);
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const float4 qv = *reinterpret_cast<const float4*>(qs + (8 * ty + r) * D + d0 + 4 * d4);
+      for (int r = 0; r < RPT; ++r) {
+        const float4 qv = *reinterpret_cast<const float4*>(qs + (RPT * ty + r) * D + d0 + 4 * d4);
         if (EST == kEstDsa2) {
           acc[r][0] += box_max_product(qv.x, qv.y, k0.x, k0.y);
           acc[r][0] += box_max_product(qv.z, qv.w, k0.z, k0.w);
@@ -330,9 +336,9 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(Geo g, SelectArg
     }
     if (d0 + kSelDChunk == D) {
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        if (j0 + tx < nb) sc[(8 * ty + r) * nb + j0 + tx] = acc[r][0] * a.scale + 0.0f;
-        if (j0 + tx + 128 < nb) sc[(8 * ty + r) * nb + j0 + tx + 128] = acc[r][1] * a.scale + 0.0f;
+      for (int r = 0; r < RPT; ++r) {
+        if (j0 + tx < nb) sc[(RPT * ty + r) * nb + j0 + tx] = acc[r][0] * a.scale + 0.0f;
+        if (j0 + tx + 128 < nb) sc[(RPT * ty + r) * nb + j0 + tx + 128] = acc[r][1] * a.scale + 0.0f;
       }
     }
     __syncthreads();   // buffer (c & 1) is refilled by the copy issued next iteration
@@ -340,7 +346,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(Geo g, SelectArg
   __syncthreads();
 
   // ---- phase 2: one warp per row: softmax statistics and selection ----
-  for (int r = warp; r < kSelRows; r += kSelThreads / 32) {
+  for (int r = warp; r < ROWS; r += kSelThreads / 32) {
     const int i = i0 + r;
     if (i >= nb) break;
     const float* row = sc + r * nb;
@@ -437,17 +443,26 @@ cudaError_t launch_intra_select(const Geo& g, const IntraArgs& a, cudaStream_t s
   return cudaGetLastError();
 }
 
-template <int D, int EST>
-static cudaError_t launch_select_t(const Geo& g, const SelectArgs& a, cudaStream_t st) {
-  const size_t smem = select_smem_bytes(g.nb, D);
+template <int D, int EST, int ROWS>
+static cudaError_t launch_select_rows(const Geo& g, const SelectArgs& a, cudaStream_t st) {
+  const size_t smem = select_smem_bytes(g.nb, D, ROWS);
   // with a head map, y enumerates its pairs (z = 1) and the kernel reads
   // map_bh(y); without one, y = h and z = b
-  dim3 grid((g.nb + kSelRows - 1) / kSelRows, a.map.n ? a.map.n : g.Hd, a.map.n ? 1 : g.B);
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<D, EST>,
+  dim3 grid((g.nb + ROWS - 1) / ROWS, a.map.n ? a.map.n : g.Hd, a.map.n ? 1 : g.B);
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<D, EST, ROWS>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  select_kernel<D, EST><<<grid, kSelThreads, smem, st>>>(g, a);
+  select_kernel<D, EST, ROWS><<<grid, kSelThreads, smem, st>>>(g, a);
   return cudaGetLastError();
+}
+
+// 16 rows per CTA while two CTAs fit on an SM; long rows (their scores fill
+// shared memory) take 8 rows per CTA so that two CTAs still fit.
+template <int D, int EST>
+static cudaError_t launch_select_t(const Geo& g, const SelectArgs& a, cudaStream_t st) {
+  constexpr size_t kTwoPerSm = 112 * 1024;
+  return select_smem_bytes(g.nb, D, kSelRows) <= kTwoPerSm ? launch_select_rows<D, EST, kSelRows>(g, a, st)
+                                                           : launch_select_rows<D, EST, 8>(g, a, st);
 }
 
 cudaError_t launch_select(const Geo& g, const SelectArgs& a, cudaStream_t st) {
