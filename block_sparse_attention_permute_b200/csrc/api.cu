@@ -431,7 +431,8 @@ bsa_status run_forward_fused(const bsa_plan_s* p, const void* q, const void* k, 
     return s;
   int32_t* sched = nullptr;
   int32_t* lists = nullptr;
-  if (pair_ws != nullptr &&
+  // pairing only reorders the work; plans beyond its block limit run unpaired
+  if (pair_ws != nullptr && bsa::pairing_supported(p->g) &&
       (s = run_pairing(p, idx, cnt, kmax, pair_ws, &sched, &lists, st, map)) != BSA_OK)
     return s;
   return run_attention_orig(p, q, k, v, idx, cnt, kmax, o, dev_status, st, map, sched, lists);
@@ -671,8 +672,6 @@ bsa_status bsa_workspace_size(bsa_plan_t p, int kmax, size_t* select_ws, size_t*
   const size_t lists = round256((size_t)p->g.B * p->g.Hd * p->g.nb * kmax * sizeof(int32_t)) +
                        round256((size_t)p->g.B * p->g.Hd * p->g.nb * sizeof(int32_t));
   if (select_ws) *select_ws = 2 * cent;
-  // The tensor-core path fuses the layout transform into the attention loads;
-  // the SIMT path stages blocked Q, K, V and O.
   // The SIMT path stages blocked Q, K, V and O; the tensor-core path fuses the
   // layout transform into the attention loads and pairs the query tiles.
   if (forward_ws)
@@ -1037,6 +1036,9 @@ bsa_status bsa_pair_tiles(bsa_plan_t p, const int32_t* idx, const int32_t* cnt, 
   if (s != BSA_OK) return s;
   if (p->attn_path != 1)
     return fail(BSA_ERR_UNSUPPORTED, "tile pairing serves bf16 plans with 128-token blocks");
+  if (!bsa::pairing_supported(p->g))
+    return fail(BSA_ERR_UNSUPPORTED, "tile pairing serves plans with at most 1536 video blocks (nb = %d)",
+                p->g.nb);
   if (kmax < 1) return fail(BSA_ERR_INVALID_ARG, "kmax must be >= 1");
   if (p->g.nb > 0 && (!idx || !cnt)) return fail(BSA_ERR_INVALID_ARG, "NULL index list");
   if (ws == nullptr || ws_bytes < pairing_bytes(p, kmax))
@@ -1054,6 +1056,9 @@ bsa_status bsa_attention_paired(bsa_plan_t p, const void* q, const void* k, cons
                                 size_t ws_bytes, void* o, int32_t* dev_status, void* stream) {
   bsa_status s = check_plan(p);
   if (s != BSA_OK) return s;
+  if (p->attn_path != 1 || !bsa::pairing_supported(p->g))
+    return fail(BSA_ERR_UNSUPPORTED, "paired attention serves bf16 plans with 128-token blocks and at "
+                                     "most 1536 video blocks");
   if (ws == nullptr || ws_bytes < pairing_bytes(p, kmax))
     return fail(BSA_ERR_WORKSPACE, "paired attention needs the %zu-byte pairing workspace, got %zu",
                 pairing_bytes(p, kmax), ws_bytes);

@@ -127,6 +127,9 @@ cudaError_t launch_select(const Geo& g, const SelectArgs& a, cudaStream_t st);
 cudaError_t launch_intra_select(const Geo& g, const IntraArgs& a, cudaStream_t st);
 // pair.cu
 size_t pair_scratch_bytes(const Geo& g);
+// Tile pairing serves plans with at most 32 * 48 = 1536 video blocks (bit sets
+// of 48 words); larger plans run the attention unpaired.
+bool pairing_supported(const Geo& g);
 cudaError_t launch_pairing(const Geo& g, const PairArgs& a, cudaStream_t st);
 // attn.cu
 size_t attn_tc_smem_bytes(int D);

@@ -23,6 +23,8 @@ constexpr int kPairRounds = 4;
 constexpr int kMaxWords = 48;   // nb <= 1536
 constexpr int kCand = 8;        // candidate partners kept per query block
 
+bool pairing_supported(const Geo& g) { return g.nb <= 32 * kMaxWords; }
+
 size_t pair_scratch_bytes(const Geo& g) {
   const size_t nbw = (g.nb + 31) / 32;
   const size_t bh = (size_t)g.B * g.Hd;

@@ -467,13 +467,16 @@ bsa_status bsa_forward_grouped(const bsa_plan_t* plans, int n_plans,
 bsa_status bsa_pair_workspace_size(bsa_plan_t plan, int kmax, size_t* bytes);
 
 /* bsa_pair_tiles — pairs the query tiles of idx / cnt ([B, Hd, nb, kmax],
- * [B, Hd, nb]) into `ws` (256-byte aligned, >= bsa_pair_workspace_size). */
+ * [B, Hd, nb]) into `ws` (256-byte aligned, >= bsa_pair_workspace_size).
+ * Serves plans with at most 1536 video blocks (BSA_ERR_UNSUPPORTED beyond;
+ * bsa_forward then runs the attention unpaired). */
 bsa_status bsa_pair_tiles(bsa_plan_t plan, const int32_t* idx,
                           const int32_t* cnt, int kmax, void* ws,
                           size_t ws_bytes, void* stream);
 
 /* bsa_attention_paired — bsa_attention_orig on the schedule bsa_pair_tiles
- * wrote into ws from the same idx / cnt. */
+ * wrote into ws from the same idx / cnt (same plan limits as
+ * bsa_pair_tiles). */
 bsa_status bsa_attention_paired(bsa_plan_t plan, const void* q, const void* k,
                                 const void* v, const int32_t* idx,
                                 const int32_t* cnt, int kmax, const void* ws,

@@ -242,3 +242,36 @@ def test_full_workload_forward(name, dev):
     got = out[:, torch.from_numpy(rows).to(dev)]
     mx, mean = check_output(to_np(got), ref, w.dtype, name)
     print(f"{name}: ties={n_tie} max_abs={mx:.3e} mean_abs={mean:.3e} rows={len(rows)}")
+
+
+def test_forward_beyond_pairing_limit(dev):
+    """A tensor-core plan with more video blocks (2048) than tile pairing serves
+    (1536): bsa_forward runs the attention unpaired and equals the explicit
+    unpaired calls bit for bit; bsa_pair_tiles refuses the plan; the lists
+    (selected with the shared-memory threshold search of long rows) match the
+    oracle and sampled output rows match the oracle's attention."""
+    w = custom_workload("many_blocks", 1, 31, 62, 126, 2, 8, 8, 1, 64, 100, "bf16", 0, 0.02)
+    g = geometry(w)
+    assert g.nb == 2048
+    (q, k, v), (qd, kd, vd) = _inputs(w, dev)
+    plan = bsa.plan_for(w, dev)
+    assert plan.info.attn_path == 1
+    out, idx, cnt = plan.forward(qd, kd, vd, w.mode, w.params, return_lists=True)
+    plan.check_status()
+    qc, kc = plan.centroids(qd, kd)
+    idx2, cnt2 = plan.select_centroids(qc, kc, w.mode, w.params)
+    out2 = plan.attention_orig(qd, kd, vd, idx2, cnt2)
+    plan.check_status()
+    assert torch.equal(cnt, cnt2) and torch.equal(idx, idx2)
+    assert torch.equal(out, out2)
+    with pytest.raises(bsa.BsaError) as e:
+        plan.pair_tiles(idx, cnt)
+    assert e.value.status == 2
+    qn, kn, vn = to_np(q), to_np(k), to_np(v)
+    p = orc.scores(g, orc.centroids(g, qn), orc.centroids(g, kn))
+    o_idx, o_cnt, tie = orc.select(g, p, w.mode, w.params)
+    check_lists(g, idx, cnt, o_idx, o_cnt, tie, p, w.mode, w.params)
+    rows = sample_rows(g, seed=7)
+    ref = orc.attention(g, qn, kn, vn, idx.cpu().numpy(), cnt.cpu().numpy(), rows=rows)
+    mx, mean = check_output(to_np(out[:, torch.from_numpy(rows).to(dev)]), ref, w.dtype, "many_blocks")
+    print(f"many_blocks: nb={g.nb} max_abs={mx:.3e} mean_abs={mean:.3e} rows={len(rows)}")
