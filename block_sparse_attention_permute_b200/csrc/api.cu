@@ -226,7 +226,7 @@ bsa_status run_select(const bsa_plan_s* p, const float* qc, const float* kc, bsa
   if (p->g.nb == 0) return BSA_OK;
   if (!qc || !kc || !idx || !cnt) return fail(BSA_ERR_INVALID_ARG, "NULL centroid or list pointer");
   if (!aligned16(qc) || !aligned16(kc)) return fail(BSA_ERR_INVALID_ARG, "summaries must be 16-byte aligned");
-  if (est != bsa::kEstMean && bsa::select_smem_bytes(p->g.nb, 2 * p->g.D) > 227 * 1024)
+  if (est != bsa::kEstMean && bsa::select_smem_bytes(p->g.nb, 2 * p->g.D, 8) > 227 * 1024)
     return fail(BSA_ERR_UNSUPPORTED, "nb = %d is too large for the box estimators", p->g.nb);
   bsa::SelectArgs a;
   std::memset(&a, 0, sizeof(a));
@@ -608,7 +608,8 @@ bsa_status bsa_plan_create(bsa_plan_t* out, int batch, int T, int H, int W, int 
   g.nb = (int)nb;
   if ((long long)batch * heads * npad >= (1ll << 31) || (long long)batch * g.n_tot * heads >= (1ll << 31))
     return fail(BSA_ERR_UNSUPPORTED, "problem exceeds 2^31 rows");
-  if (bsa::select_smem_bytes(g.nb, head_dim) > 227 * 1024)
+  // the selection kernel takes 8 query rows per CTA when 16 do not fit twice
+  if (bsa::select_smem_bytes(g.nb, head_dim, 8) > 227 * 1024)
     return fail(BSA_ERR_UNSUPPORTED, "nb = %d video blocks exceeds the selection kernel's limit", g.nb);
   p.dtype = dtype;
   p.attn_path = (dtype == BSA_BF16 && bs == 128) ? 1 : 0;
