@@ -602,11 +602,7 @@ def run_ours(args, rank, world, local):
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
         "config": {
-            "workload": w.name,
-            "shape": f"grid {w.T}x{w.H}x{w.W} + {w.n_text} text, block {w.bf}x{w.br}x{w.bc}, "
-                     f"{w.Hd} heads, head_dim {w.D}, batch {w.B}",
-            "selection": ("top-k density " if w.mode == 0 else "top-p tau ") +
-                         (str(w.params[0]) if len(set(w.params)) == 1 else "per-head mix"),
+            **workload_config(w),
             "parallelism": f"replicas x{world} (no collective)",
             "l2": f"inputs {3 * q.numel() * q.element_size() / 1e9:.2f} GB > 126 MB L2 (no flush)",
             "effective_tflop_per_step": round(flops / 1e12, 4),
@@ -654,6 +650,17 @@ def run_ours(args, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
+def workload_config(w):
+    """The workload keys shared by both arms' config."""
+    return {
+        "workload": w.name,
+        "shape": f"grid {w.T}x{w.H}x{w.W} + {w.n_text} text, block {w.bf}x{w.br}x{w.bc}, "
+                 f"{w.Hd} heads, head_dim {w.D}, batch {w.B}",
+        "selection": ("top-k density " if w.mode == 0 else "top-p tau ") +
+                     (str(w.params[0]) if len(set(w.params)) == 1 else "per-head mix"),
+    }
+
+
 def cpu_baseline(w, q, k, v, budget_s=20.0):
     """The fp64 oracle, as it stands, on a bounded sample of the workload."""
     import oracle as orc
@@ -690,7 +697,9 @@ def cpu_baseline(w, q, k, v, budget_s=20.0):
             break
     flops = 4.0 * pairs * g.D
     tf = flops / t_att / 1e12
+    full_flop = 4.0 * orc.selected_pairs(g, idx, cnt) * g.D
     return {"value": tf, "unit": "TFLOP/s", "cores": orc.threads(), "kind": "oracle",
+            "full_step_flop": full_flop,
             "sample": f"oracle centroids+scores+selection on the full workload ({t_sel:.1f} s), "
                       f"attention on {nblk} random query blocks x all {g.Hd} heads "
                       f"({t_att:.1f} s); value = effective FLOP of the sampled attention / its time"}
@@ -716,12 +725,17 @@ def run_reference(args, rank, world):
             vals.append(cb["value"])
     value = float(np.mean(vals))
     cb["value"] = value
+    # one whole step of the workload at the sampled rate
+    ms_full = cb["full_step_flop"] / (value * 1e12) * 1e3
+    config = workload_config(w)
+    config["parallelism"] = f"host cores ({cb['cores']} oracle threads)"
+    config["ms_per_step_note"] = "one full step extrapolated from the sampled rate"
     line = {
         "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_full, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": w.name, "parallelism": "host cores (oracle threads)"},
+        "config": config,
         "cpu_baseline": cb,
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
