@@ -61,10 +61,16 @@ def peaks():
 
 
 def attn_source_sha() -> str:
+    """Hash of the attention kernel's code: its sources with // comments and
+    whitespace removed (none of them has // inside a string literal), so that
+    an edit to a comment does not void a profile taken on the same code."""
     h = hashlib.sha256()
     for name in ("attn.cu", "common.cuh", "kernels.cuh"):
-        with open(os.path.join(ROOT, "block_sparse_attention_permute_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "block_sparse_attention_permute_b200", "csrc", name)) as f:
+            for line in f:
+                code = "".join(line.split("//", 1)[0].split())
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -8,14 +8,16 @@
 // memory/compute".  The per-query-block index lists are the sparse rows.
 //
 // Two kernels:
-//  * attn_tc_kernel (bf16, 128-token blocks, D in {64,128}): one CTA per
-//    (batch, head, query block).  Warp 4 issues TMA loads of Q once and of
-//    the K/V tiles of the selected key blocks only (two stages); warp 5 issues
-//    tcgen05.mma: S = Q K^T into TMEM, O += P V into TMEM; warps 0-3 own one
-//    query row per thread: they read S from TMEM, apply the pad mask and the
-//    online softmax (exp2 of log2e-prescaled logits, fp32 statistics),
-//    rescale O in TMEM when the running max grows, and write P (bf16) to
-//    shared memory for the PV product.  The epilogue divides by the row sum.
+//  * attn_tc_kernel (bf16, 128-token blocks, D in {64,128}): one CTA per two
+//    query tiles (a pair of the tile-pairing schedule, or two consecutive
+//    tiles); warp 8 issues TMA loads of the two Q tiles once and of the K/V
+//    tiles of the selected key blocks only, through a 4-slot ring; warp 9
+//    issues tcgen05.mma: S = Q K^T into TMEM, O += P V into TMEM, P read
+//    from TMEM; warps 0-3 and 4-7 own one query row per thread of tile 0 and
+//    tile 1: they read S from TMEM, apply the pad mask and the online softmax
+//    (exp2 of log2e-prescaled logits, fp32 statistics, lazy rescaling of O in
+//    TMEM), and write P (bf16) back into TMEM for the PV product.  The
+//    epilogue divides by the row sum.  Details at the kernel.
 //  * attn_simt_kernel (any dtype, any block size <= 256): one warp per query
 //    row, fp32 scores and online softmax, exact fp32 arithmetic.  It serves
 //    fp32 inputs and block shapes the tensor-core path does not take.

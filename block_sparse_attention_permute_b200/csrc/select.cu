@@ -10,9 +10,9 @@
 // in ascending order, so the value does not depend on the launch shape);
 // p_ij = e_ij / Z_i with e_ij = expf(s_ij - max_j s_ij) and Z_i summed in fp64.
 // Selection, one warp per query-block row:
-//   Top-K: the k-th largest score is found by a 32-step bitwise search over
-//          the order-preserving integer image of s; equal scores are taken in
-//          ascending block id.
+//   Top-K: the k-th largest score is found by a bitwise search (at most 32
+//          steps) over the order-preserving integer image of s; equal scores
+//          are taken in ascending block id.
 //   Top-P: the largest score threshold whose mass sum_{s_j >= t} e_j reaches
 //          tau * Z (fp64), then ties at the threshold in ascending block id
 //          until the mass is reached: the shortest prefix in descending order.
