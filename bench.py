@@ -591,6 +591,7 @@ def run_ours(args, rank, world, local):
     if rank != 0:
         return
     peak_tf, hbm_gbs, peak_src = peaks()
+    phase_roof = phase_rooflines(w, plan, fused, unfused, hbm_gbs)
     value = job_tflops(world, flops, step_ms)
     attn_tf = flops / (attn_ms * 1e-3) / 1e12
     traffic = profiled_traffic(args.workload)
@@ -618,6 +619,7 @@ def run_ours(args, rank, world, local):
         "phases_ms_unfused": {n: round(t, 4) for n, t in unfused.items()},
         "attn_tflops": round(attn_tf, 2),
         "attn_frac_of_peak": round(attn_tf / peak_tf, 4),
+        "phase_rooflines": phase_roof,
         "permute_select_share_of_attn": round(
             (phase_ms.get("centroids", phase_ms.get("permute", 0.0)) + phase_ms["select"]
              + phase_ms.get("pairing", 0.0)) / phase_ms["attention"], 4),
@@ -654,6 +656,44 @@ def run_ours(args, rank, world, local):
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, q, k, v, budget_s=args.cpu_seconds)
     print(json.dumps(line), flush=True)
+
+
+# fp32 FMA peak of the selection's score GEMM: 148 SMs x 128 FMA lanes x 2 FLOP
+# x the 1965 MHz maximum SM clock (derived from the unit counts, not measured)
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def phase_rooflines(w, plan, fused, unfused, hbm_gbs):
+    """Achieved rate of every non-attention phase against its roofline, from
+    the phases' CUDA-event times: HBM phases by their algorithmic bytes (each
+    input byte read once, each output byte written once), the selection by the
+    fp32 FLOP of its score GEMM."""
+    e = 2 if w.dtype == "bf16" else 4
+    info = plan.info
+    row = w.Hd * w.D * e * w.B                       # bytes of one token of Q, K or V
+    n_tot, n_pad = info.n_tot, info.npad_tot
+    cent_out = 2 * w.B * w.Hd * info.nb * w.D * 4
+    out = {}
+
+    def hbm(name, ms, nbytes):
+        if ms and ms > 0:
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            out[name] = {"bound": "hbm", "bytes": int(nbytes), "ms": round(ms, 4),
+                         "achieved_gbs": round(gbs, 1), "peak_gbs": hbm_gbs,
+                         "frac": round(gbs / hbm_gbs, 3)}
+
+    if fused is not None:
+        hbm("centroids", fused["centroids"], 2 * info.n_video * row + cent_out)   # video tokens only
+    hbm("permute_qkv", unfused["permute"], 3 * n_tot * row + 3 * n_pad * row + cent_out)
+    hbm("unpermute", unfused["unpermute"], n_pad * row + n_tot * row)
+    sel_ms = (fused or unfused)["select"]
+    sel_flop = 2.0 * w.B * w.Hd * info.nb * info.nb * w.D
+    tf = sel_flop / (sel_ms * 1e-3) / 1e12
+    out["select"] = {"bound": "alu", "flop": sel_flop, "ms": round(sel_ms, 4),
+                     "achieved_tflops": round(tf, 2), "peak_tflops": round(FP32_PEAK_TFLOPS, 1),
+                     "peak_source": "derived: 148 SMs x 128 fp32 FMA/clk x 2 x 1965 MHz",
+                     "frac": round(tf / FP32_PEAK_TFLOPS, 3)}
+    return out
 
 
 def workload_config(w):
