@@ -275,3 +275,29 @@ def test_forward_beyond_pairing_limit(dev):
     ref = orc.attention(g, qn, kn, vn, idx.cpu().numpy(), cnt.cpu().numpy(), rows=rows)
     mx, mean = check_output(to_np(out[:, torch.from_numpy(rows).to(dev)]), ref, w.dtype, "many_blocks")
     print(f"many_blocks: nb={g.nb} max_abs={mx:.3e} mean_abs={mean:.3e} rows={len(rows)}")
+
+
+# Row lengths the other cases do not reach: 600 blocks (the register search
+# with 32 keys per lane, Top-K and Top-P) and 1100 blocks with Top-P (the
+# shared-memory mass search; Top-K keeps 48 keys per lane in registers there).
+ROW_CASES = {
+    "mid_topk": (custom_workload("mid_topk", 1, 24, 40, 80, 1, 8, 16, 2, 64, 0, "bf16", 0, 0.1), 600),
+    "mid_topp": (custom_workload("mid_topp", 1, 24, 40, 80, 1, 8, 16, 2, 64, 0, "bf16", 1, 0.8), 600),
+    "long_topp": (custom_workload("long_topp", 1, 44, 40, 80, 1, 8, 16, 1, 64, 0, "bf16", 1, 0.8), 1100),
+}
+
+
+@pytest.mark.parametrize("name", list(ROW_CASES))
+def test_select_long_rows(name, dev):
+    w, nb = ROW_CASES[name]
+    g = geometry(w)
+    assert g.nb == nb
+    (q, k, _), (qd, kd, _) = _inputs(w, dev)
+    plan = bsa.plan_for(w, dev)
+    qc, kc = plan.centroids(qd, kd)
+    idx, cnt = plan.select_centroids(qc, kc, w.mode, w.params)
+    plan.check_status()
+    p = orc.scores(g, orc.centroids(g, to_np(q)), orc.centroids(g, to_np(k)))
+    o_idx, o_cnt, tie = orc.select(g, p, w.mode, w.params)
+    n_tie = check_lists(g, idx, cnt, o_idx, o_cnt, tie, p, w.mode, w.params)
+    print(f"{name}: nb={g.nb} ties={n_tie} mean list {float(cnt.float().mean()):.1f}")
