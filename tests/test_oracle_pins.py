@@ -324,6 +324,20 @@ def test_sics_special_cases():
     assert abs(orc.sics_online(g, x)[0, 1, 0] - 7.0) < 1e-12
 
 
+def test_kmax_for_bounds_the_lists():
+    # the list width is the longest list the selection can produce: Top-K lists
+    # have exactly k_h + nb_text entries, so the widest reaches it; Top-P lists
+    # never exceed it
+    g = orc.Geometry(B=2, T=4, H=8, W=12, bf=2, br=4, bc=4, Hd=3, D=16, n_text=40)
+    q, k = rand_x(g, 5), rand_x(g, 6)
+    p = orc.scores(g, orc.centroids(g, q), orc.centroids(g, k))
+    dens = [0.1, 0.35, 0.6]
+    _, cnt, _ = orc.select(g, p, 0, dens)
+    assert orc.kmax_for(g, 0, dens) == int(cnt.max())
+    _, cnt, _ = orc.select(g, p, 1, [0.5, 0.9, 1.0])
+    assert int(cnt.max()) <= orc.kmax_for(g, 1, [0.5, 0.9, 1.0])
+
+
 def test_aggregation_score_and_scheme_choice():
     # AS = sum of block SICS (Eq. (3)); the chosen scheme maximises it
     base = dict(B=1, T=4, H=8, W=8, Hd=3, D=16, n_text=0)
