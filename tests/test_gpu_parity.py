@@ -301,3 +301,34 @@ def test_select_long_rows(name, dev):
     o_idx, o_cnt, tie = orc.select(g, p, w.mode, w.params)
     n_tie = check_lists(g, idx, cnt, o_idx, o_cnt, tie, p, w.mode, w.params)
     print(f"{name}: nb={g.nb} ties={n_tie} mean list {float(cnt.float().mean()):.1f}")
+
+
+@pytest.mark.parametrize("name", ["hy_ragged_text", "wan_d64_b2", "f32_bs128"])
+def test_forward_in_cuda_graph(name, dev):
+    """bsa_forward makes no synchronous CUDA call after plan creation, so it can
+    be captured in a CUDA graph: replays on fresh inputs equal eager calls
+    bit for bit (tensor-core plans, with pairing, and the fp32 SIMT path)."""
+    w = SMALL[name]
+    (_, _, _), (qd, kd, vd) = _inputs(w, dev)
+    plan = bsa.plan_for(w, dev)
+    kmax = plan.kmax_for(w.mode, w.params)
+    ws = torch.empty(plan.workspace_size(kmax)[1], dtype=torch.uint8, device=dev)
+    qs, ks, vs, out = qd.clone(), kd.clone(), vd.clone(), torch.empty_like(qd)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):   # warm-up outside the capture
+        plan.forward(qs, ks, vs, w.mode, w.params, kmax=kmax, out=out, workspace=ws)
+    torch.cuda.current_stream(dev).wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        plan.forward(qs, ks, vs, w.mode, w.params, kmax=kmax, out=out, workspace=ws)
+    for scale in (1.0, 0.5):
+        qs.copy_(qd * scale)
+        ks.copy_(kd)
+        vs.copy_(vd * (2.0 - scale))
+        graph.replay()
+        eager = plan.forward(qs, ks, vs, w.mode, w.params, kmax=kmax)
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager)
+    plan.check_status()
+    del graph
