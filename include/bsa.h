@@ -41,11 +41,10 @@
  *    every key block (dense rows).  Text blocks take no part in scoring.
  *  - Errors: every call returns a bsa_status; bsa_last_error_string() gives a
  *    thread-local message for the last failure.
- *  - After bsa_plan_create, the compute calls (bsa_permute .. bsa_forward_*)
- *    make no synchronous CUDA call and allocate nothing, so they can be
- *    captured in a CUDA graph; per-head parameters are read on the host at
- *    the call (at capture) and travel in the kernel arguments.  Only
- *    bsa_check_status synchronises.
+ *  - bsa_forward makes no synchronous CUDA call and allocates nothing (the
+ *    caller passes the workspace), so it can be captured in a CUDA graph;
+ *    its per-head parameters are read on the host at the call (at capture)
+ *    and travel in the kernel arguments.  bsa_check_status synchronises.
  */
 #ifndef BSA_H_
 #define BSA_H_
