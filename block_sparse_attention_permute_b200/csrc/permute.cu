@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(Geo g, GatherArg
 // threads per (tensor, block j, group of heads); thread (head, v) owns the
 // 16-byte column v of one head and streams it through the block's 128 slots,
 // so a warp reads whole runs of adjacent heads of one token and no partial
-// sums cross threads.  The sums are formed in the order of gather_block's
+// sums cross threads (M = 128 / R independent 16-byte loads per row group).  The sums are formed in the order of gather_block's
 // kPool path (row group r = s mod R holds s = r, r + R, ...; the groups are
 // then added in ascending r), so the centroids are bit-identical to the
 // blocked-layout pool.
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(kColThreads) pool_cols_kernel(Geo g, GatherArg
   float total[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) total[e] = 0.f;
-#pragma unroll 2
+#pragma unroll 1   // 64 registers: 8 CTAs per SM keep more loads in flight than a deeper unroll
   for (int r = 0; r < R; ++r) {
     uint4 x[M];
     int tok[M];
