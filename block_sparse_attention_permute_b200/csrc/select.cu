@@ -24,14 +24,14 @@ namespace bsa {
 
 constexpr int kSelRows = 16;      // query-block rows per CTA (8 for long rows, see launch_select_t)
 constexpr int kSelKeys = 256;     // key blocks per score chunk
-constexpr int kSelDChunk = 16;    // head-dim slice of a key chunk held in shared memory
+constexpr int kSelDChunk = 8;    // head-dim slice of a key chunk held in shared memory
+constexpr int kSelBufs = 2;      // key-chunk buffers (2: the next chunk lands while one is used)
 constexpr int kSelKS = kSelDChunk + 4;   // padded chunk row: conflict-free float4 reads
 constexpr int kSelThreads = 256;  // 8 warps
 
-// query summaries, two key-chunk buffers (the next chunk lands while the
-// current one is used), the score rows
+// query summaries, the key-chunk buffers, the score rows
 size_t select_smem_bytes(int nb, int D, int rows) {
-  return sizeof(float) * ((size_t)rows * D + 2 * (size_t)kSelKeys * kSelKS + (size_t)rows * nb);
+  return sizeof(float) * ((size_t)rows * D + kSelBufs * (size_t)kSelKeys * kSelKS + (size_t)rows * nb);
 }
 
 __device__ __forceinline__ uint32_t order_key(float s) {
@@ -164,7 +164,11 @@ __device__ __forceinline__ void rule_threshold_regs(const float* row, int nb, in
 // with key == T.  Top-K: param = k.  Top-P: param = tau, `total` = the sum of
 // all weights; the shortest descending prefix whose weight reaches
 // tau * total (at least one entry).
-template <class Wt>
+// KMAX: the most keys per lane this instance keeps in registers (0: none,
+// every row takes the shared-memory loops); the launch picks the smallest
+// that covers its rows, so short rows do not pay for the registers of long
+// ones.
+template <int KMAX, class Wt>
 __device__ __forceinline__ void rule_threshold(const float* row, int nb, int mode, double param,
                                                double total, Wt wt, int lane, uint32_t* T_out,
                                                int* need_out) {
@@ -177,17 +181,31 @@ __device__ __forceinline__ void rule_threshold(const float* row, int nb, int mod
   }
   // Registers: Top-K keeps up to 48 keys per lane, Top-P up to 32 keys and
   // their weights; longer rows use the shared-memory loops.
-  if (mode == 0 && nb <= 32 * kKeysPerLane) {
-    const int k = (int)param;
-    if (nb <= 32 * 16) rule_threshold_regs<16, false>(row, nb, k, target, wt, lane, T_out, need_out);
-    else if (nb <= 32 * 32) rule_threshold_regs<32, false>(row, nb, k, target, wt, lane, T_out, need_out);
-    else rule_threshold_regs<kKeysPerLane, false>(row, nb, k, target, wt, lane, T_out, need_out);
-    return;
+  if constexpr (KMAX >= 16) {
+    if (mode == 0 && nb <= 32 * 16) {
+      rule_threshold_regs<16, false>(row, nb, (int)param, target, wt, lane, T_out, need_out);
+      return;
+    }
+    if (mode != 0 && nb <= 32 * 16) {
+      rule_threshold_regs<16, true>(row, nb, 0, target, wt, lane, T_out, need_out);
+      return;
+    }
   }
-  if (mode != 0 && nb <= 32 * 32) {
-    if (nb <= 32 * 16) rule_threshold_regs<16, true>(row, nb, 0, target, wt, lane, T_out, need_out);
-    else rule_threshold_regs<32, true>(row, nb, 0, target, wt, lane, T_out, need_out);
-    return;
+  if constexpr (KMAX >= 32) {
+    if (mode == 0 && nb <= 32 * 32) {
+      rule_threshold_regs<32, false>(row, nb, (int)param, target, wt, lane, T_out, need_out);
+      return;
+    }
+    if (mode != 0 && nb <= 32 * 32) {
+      rule_threshold_regs<32, true>(row, nb, 0, target, wt, lane, T_out, need_out);
+      return;
+    }
+  }
+  if constexpr (KMAX >= kKeysPerLane) {
+    if (mode == 0 && nb <= 32 * kKeysPerLane) {
+      rule_threshold_regs<kKeysPerLane, false>(row, nb, (int)param, target, wt, lane, T_out, need_out);
+      return;
+    }
   }
   if (mode == 0) {
     const int k = (int)param;
@@ -236,13 +254,14 @@ __device__ __forceinline__ float box_max_product(float aM, float am, float bM, f
 
 // D = length of the stored summary vectors (head_dim for MEAN, 2 * head_dim
 // for the (max, min) boxes of DSA and DSA2).
-template <int D, int EST, int ROWS>
-__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(Geo g, SelectArgs a) {
+template <int D, int EST, int ROWS, int KMAX>
+__global__ void __launch_bounds__(kSelThreads, KMAX == 16 ? 3 : 2)
+    select_kernel(Geo g, SelectArgs a) {
   constexpr int RPT = ROWS / 2;                     // rows per thread in phase 1
   extern __shared__ __align__(16) float sm[];
   float* qs = sm;                                   // [ROWS][D]
-  float* ks = qs + ROWS * D;                        // [2][kSelKeys][kSelKS]
-  float* sc = ks + 2 * kSelKeys * kSelKS;           // [ROWS][nb]
+  float* ks = qs + ROWS * D;                        // [kSelBufs][kSelKeys][kSelKS]
+  float* sc = ks + kSelBufs * kSelKeys * kSelKS;    // [ROWS][nb]
   const int nb = g.nb;
   const int bhi = map_bh(a.map, (int)blockIdx.z * g.Hd + (int)blockIdx.y);
   const int h = bhi % g.Hd, b = bhi / g.Hd;
@@ -252,7 +271,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(Geo g, SelectArg
 
   // ---- phase 1: scores of ROWS query blocks against all key blocks ----
   // Thread (ty, tx) accumulates rows RPT ty .. RPT ty + RPT - 1 against keys tx and tx+128 of
-  // each 256-key chunk; the chunk's keys pass through shared memory 16
+  // each 256-key chunk; the chunk's keys pass through shared memory 8
   // dimensions at a time (double-buffered).  Each dot product is one fma chain over d in
   // ascending order, the same as a plain sequential loop.
   if (EST == kEstDsa) {
@@ -285,7 +304,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(Geo g, SelectArg
   const float* kc_bh = a.kc + bh * nb * D;
   auto issue_chunk = [&](int c) {
     const int j0 = (c / kDChunks) * kSelKeys, d0 = (c % kDChunks) * kSelDChunk;
-    float* buf = ks + (c & 1) * kSelKeys * kSelKS;
+    float* buf = ks + (c % kSelBufs) * kSelKeys * kSelKS;
     for (int e = tid; e < kSelKeys * (kSelDChunk / 4); e += kSelThreads) {
       const int jj = e / (kSelDChunk / 4), d4 = e % (kSelDChunk / 4);
       const bool ok = j0 + jj < nb;
@@ -294,7 +313,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(Geo g, SelectArg
     }
     cp_async_commit();
   };
-  issue_chunk(0);
+  if (kSelBufs == 2) issue_chunk(0);
   float acc[RPT][2];
   for (int c = 0; c < n_chunks; ++c) {
     const int j0 = (c / kDChunks) * kSelKeys, d0 = (c % kDChunks) * kSelDChunk;
@@ -302,14 +321,17 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(Geo g, SelectArg
 #pragma unroll
       for (int r = 0; r < RPT; ++r) acc[r][0] = acc[r][1] = 0.f;
     }
-    if (c + 1 < n_chunks) {
+    if (kSelBufs == 1) {
+      issue_chunk(c);
+      cp_async_wait<0>();
+    } else if (c + 1 < n_chunks) {
       issue_chunk(c + 1);
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
     }
     __syncthreads();   // chunk c (and, at c = 0, the query summaries) visible
-    const float* kb = ks + (c & 1) * kSelKeys * kSelKS;
+    const float* kb = ks + (c % kSelBufs) * kSelKeys * kSelKS;
 #pragma unroll
     for (int d4 = 0; d4 < kSelDChunk / 4; ++d4) {
       const float4 k0 = *reinterpret_cast<const float4*>(kb + tx * kSelKS + 4 * d4);
@@ -366,7 +388,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(Geo g, SelectArg
 
     uint32_t T = 0;
     int need = 0;  // how many of the scores equal to the threshold to take
-    rule_threshold(row, nb, a.mode, a.param[h], Z, SoftmaxWeight{m}, lane, &T, &need);
+    rule_threshold<KMAX>(row, nb, a.mode, a.param[h], Z, SoftmaxWeight{m}, lane, &T, &need);
 
     // Ascending compaction of {key > T} plus the first `need` of {key == T},
     // united with the window, sink and intra blocks.
@@ -420,7 +442,7 @@ __global__ void __launch_bounds__(kIntraWarps * 32) intra_select_kernel(Geo g, I
   const double total = a.mode != 0 ? mass_at_least(row, nb, PlainWeight{}, 0u, lane) : 0.0;
   uint32_t T = 0;
   int need = 0;
-  rule_threshold(row, nb, a.mode, prm, total, PlainWeight{}, lane, &T, &need);
+  rule_threshold<kKeysPerLane>(row, nb, a.mode, prm, total, PlainWeight{}, lane, &T, &need);
   int eq_seen = 0;
   const uint32_t lt_mask = (1u << lane) - 1u;
   for (int j0 = 0; j0 < nb; j0 += 32) {
@@ -443,26 +465,34 @@ cudaError_t launch_intra_select(const Geo& g, const IntraArgs& a, cudaStream_t s
   return cudaGetLastError();
 }
 
-template <int D, int EST, int ROWS>
+template <int D, int EST, int ROWS, int KMAX>
 static cudaError_t launch_select_rows(const Geo& g, const SelectArgs& a, cudaStream_t st) {
   const size_t smem = select_smem_bytes(g.nb, D, ROWS);
   // with a head map, y enumerates its pairs (z = 1) and the kernel reads
   // map_bh(y); without one, y = h and z = b
   dim3 grid((g.nb + ROWS - 1) / ROWS, a.map.n ? a.map.n : g.Hd, a.map.n ? 1 : g.B);
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<D, EST, ROWS>,
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<D, EST, ROWS, KMAX>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  select_kernel<D, EST, ROWS><<<grid, kSelThreads, smem, st>>>(g, a);
+  select_kernel<D, EST, ROWS, KMAX><<<grid, kSelThreads, smem, st>>>(g, a);
   return cudaGetLastError();
 }
 
-// 16 rows per CTA while two CTAs fit on an SM; long rows (their scores fill
-// shared memory) take 8 rows per CTA so that two CTAs still fit.
+// Rows of up to 512 / 1024 / 1536 key blocks keep 16 / 32 / 48 keys per lane
+// in registers (16 keys fit in 80 registers: three CTAs per SM), longer rows
+// none.  16 query rows per CTA while two CTAs fit on an SM; long rows (their
+// scores fill shared memory) take 8 rows per CTA so that two CTAs still fit.
 template <int D, int EST>
 static cudaError_t launch_select_t(const Geo& g, const SelectArgs& a, cudaStream_t st) {
   constexpr size_t kTwoPerSm = 112 * 1024;
-  return select_smem_bytes(g.nb, D, kSelRows) <= kTwoPerSm ? launch_select_rows<D, EST, kSelRows>(g, a, st)
-                                                           : launch_select_rows<D, EST, 8>(g, a, st);
+  const bool rows16 = select_smem_bytes(g.nb, D, kSelRows) <= kTwoPerSm;
+  if (g.nb <= 32 * 16 && rows16) return launch_select_rows<D, EST, kSelRows, 16>(g, a, st);
+  if (g.nb <= 32 * 32 && rows16) return launch_select_rows<D, EST, kSelRows, 32>(g, a, st);
+  if (g.nb <= 32 * kKeysPerLane)
+    return rows16 ? launch_select_rows<D, EST, kSelRows, kKeysPerLane>(g, a, st)
+                  : launch_select_rows<D, EST, 8, kKeysPerLane>(g, a, st);
+  return rows16 ? launch_select_rows<D, EST, kSelRows, 0>(g, a, st)
+                : launch_select_rows<D, EST, 8, 0>(g, a, st);
 }
 
 cudaError_t launch_select(const Geo& g, const SelectArgs& a, cudaStream_t st) {
