@@ -270,6 +270,109 @@ __global__ void __launch_bounds__(kColThreads) pool_cols_kernel(Geo g, GatherArg
   out[1] = make_float4(total[4] / n, total[5] / n, total[6] / n, total[7] / n);
 }
 
+// The same pass with the optional outputs of the mask unions and the box
+// estimators: (max, min) per dimension over the block's valid rows (exact in
+// any order) and the SICS of SPADE §3.2 Eq. (4) as || sum_a x_a / |x_a| ||^2
+// (a zero row has no direction and adds nothing).  A row's squared norm is
+// summed over the V lanes that hold it (an aligned lane group of the warp);
+// the unit rows are accumulated in the centroid's group order.  Threads past
+// the last head still run the loop on the last head (their lanes take part
+// in the shuffles) and store nothing.
+template <int D>
+__global__ void __launch_bounds__(kColThreads) pool_cols_extras_kernel(Geo g, GatherArgs a) {
+  using T = __nv_bfloat16;
+  constexpr int E = 8;                      // bf16 elements per 16-byte vector
+  constexpr int V = D / E;                  // vectors per row (lanes per row)
+  constexpr int R = kGatherThreads / V;     // row groups, as in gather_block
+  constexpr int M = 128 / R;                // rows per group
+  constexpr int HG = kColThreads / V;       // heads per CTA
+  __shared__ int s_tok[128];
+  const int j = blockIdx.x, t = blockIdx.z;
+  const int pairs = map_count(a.map, g.B * g.Hd);
+  const int p_raw = blockIdx.y * HG + (int)threadIdx.x / V, vec = (int)threadIdx.x % V;
+  const bool active = p_raw < pairs;
+  const int p = active ? p_raw : pairs - 1;
+  const void* src_ptr = t == 0 ? a.src[0] : t == 1 ? a.src[1] : a.src[2];
+  float* cent = t == 0 ? a.cent[0] : t == 1 ? a.cent[1] : a.cent[2];
+  float* sics = t == 0 ? a.sics[0] : t == 1 ? a.sics[1] : a.sics[2];
+  float* box = t == 0 ? a.box[0] : t == 1 ? a.box[1] : a.box[2];
+  s_tok[threadIdx.x] = (int)slot_token(g, j, threadIdx.x);
+  __syncthreads();
+  const int bh = map_bh(a.map, p), b = bh / g.Hd, h = bh % g.Hd;
+  const uint4* src = reinterpret_cast<const uint4*>(src_ptr) + ((long long)b * g.n_tot * g.Hd + h) * V + vec;
+  const long long tok_stride = (long long)g.Hd * V;   // uint4 per token
+  const bool do_sics = sics != nullptr;               // the same for the whole CTA
+  float total[E], rtot[E], bmax[E], bmin[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    total[e] = rtot[e] = 0.f;
+    bmax[e] = -INFINITY;
+    bmin[e] = INFINITY;
+  }
+#pragma unroll 1
+  for (int r = 0; r < R; ++r) {
+    uint4 x[M];
+    int tok[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      tok[m] = s_tok[r + R * m];
+      x[m] = tok[m] >= 0 ? __ldg(src + tok[m] * tok_stride) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float part[E], rpart[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) part[e] = rpart[e] = 0.f;
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      if (tok[m] < 0) continue;   // a pad slot: the same for every thread of the CTA
+      float f[E];
+      to_float<T>(x[m], f);
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        part[e] += f[e];
+        bmax[e] = fmaxf(bmax[e], f[e]);
+        bmin[e] = fminf(bmin[e], f[e]);
+      }
+      if (do_sics) {
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) ss = fmaf(f[e], f[e], ss);
+#pragma unroll
+        for (int o = V / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) rpart[e] = fmaf(f[e], inv, rpart[e]);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      total[e] += part[e];
+      rtot[e] += rpart[e];
+    }
+  }
+  float sq = 0.f;
+  if (do_sics) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) sq = fmaf(rtot[e], rtot[e], sq);
+#pragma unroll
+    for (int o = V / 2; o >= 1; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  }
+  if (!active) return;
+  const long long blk = (long long)bh * g.nb + j;
+  if (cent != nullptr) {
+    const float n = (float)block_valid_count(g, j);
+    float4* out = reinterpret_cast<float4*>(cent + blk * D + vec * E);
+    out[0] = make_float4(total[0] / n, total[1] / n, total[2] / n, total[3] / n);
+    out[1] = make_float4(total[4] / n, total[5] / n, total[6] / n, total[7] / n);
+  }
+  if (box != nullptr) {
+    float4* out = reinterpret_cast<float4*>(box + (blk * D + vec * E) * 2);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      out[q] = make_float4(bmax[2 * q], bmin[2 * q], bmax[2 * q + 1], bmin[2 * q + 1]);
+  }
+  if (do_sics && vec == 0) sics[blk] = sq;
+}
+
 // Aggregation evaluation (SPADE §3.2): SICS of every block of every candidate
 // blocking scheme, read from the original layout.  One warp per (b, h,
 // candidate, block): the online form of Eq. (5), a running sum of unit rows
@@ -453,13 +556,18 @@ cudaError_t launch_unpermute(const Geo& g, bool is_bf16, const GatherArgs& a, cu
 cudaError_t launch_pool_orig(const Geo& g, bool is_bf16, const GatherArgs& a, cudaStream_t st) {
   bool extras = false;
   for (int t = 0; t < a.ntensors; ++t) extras = extras || a.sics[t] != nullptr || a.box[t] != nullptr;
-  if (is_bf16 && g.bs == 128 && !extras && (g.D == 128 || g.D == 64)) {
+  if (is_bf16 && g.bs == 128 && (g.D == 128 || g.D == 64)) {
     const int pairs = map_count(a.map, g.B * g.Hd);
     const int hg = kColThreads / (g.D / 8);
     const dim3 grid(g.nb, (pairs + hg - 1) / hg, a.ntensors);
     if (g.nb == 0 || pairs == 0) return cudaSuccess;
-    if (g.D == 128) pool_cols_kernel<128><<<grid, kColThreads, 0, st>>>(g, a);
-    else pool_cols_kernel<64><<<grid, kColThreads, 0, st>>>(g, a);
+    if (extras) {
+      if (g.D == 128) pool_cols_extras_kernel<128><<<grid, kColThreads, 0, st>>>(g, a);
+      else pool_cols_extras_kernel<64><<<grid, kColThreads, 0, st>>>(g, a);
+    } else {
+      if (g.D == 128) pool_cols_kernel<128><<<grid, kColThreads, 0, st>>>(g, a);
+      else pool_cols_kernel<64><<<grid, kColThreads, 0, st>>>(g, a);
+    }
     return cudaGetLastError();
   }
   return is_bf16 ? launch_gather_t<__nv_bfloat16, kPoolOrig>(g, a, g.nb, st)
