@@ -439,17 +439,23 @@ def run_ours(args, rank, world, local):
 
     # ---- main timed loop: K whole steps
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev_step = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier()
     with ClockSampler(local) as clk:
         clk.mark_start()
         ev0.record(stream)
-        for _ in range(args.steps):
+        for i in range(args.steps):
             forward()
+            ev_step[i].record(stream)
         ev1.record(stream)
         barrier()
         clk.mark_end()
     plan.check_status()
     step_ms = ev0.elapsed_time(ev1) / args.steps
+    per_step = [ev0.elapsed_time(ev_step[0])] + [ev_step[i - 1].elapsed_time(ev_step[i])
+                                                for i in range(1, args.steps)]
+    step_stats = {"min": round(min(per_step), 4), "median": round(statistics.median(per_step), 4),
+                  "max": round(max(per_step), 4)}
     clocks = clk.summary()
 
     # ---- phase loops (CUDA events on the launching stream)
@@ -603,6 +609,7 @@ def run_ours(args, rank, world, local):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(step_ms, 4),
+        "ms_per_step_stats": step_stats,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,

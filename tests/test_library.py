@@ -68,13 +68,15 @@ def test_plan_validation_rejects_bad_arguments(lib, args, needle):
 
 def test_plan_block_count_limit(lib):
     # the selection kernel holds 8 score rows of nb floats per CTA (8 query
-    # rows per CTA once 16 no longer fit twice on an SM): up to 5856 blocks at
-    # head_dim 128; beyond that the plan is refused before any device work
-    st, msg = _create(lib, 1, 1, 1, 5857, 1, 1, 1, 1, 128, 0, 1)
+    # rows per CTA once 16 no longer fit twice on an SM) beside 8 query
+    # summaries and two 256 x 12-float key chunks: up to 6368 blocks at
+    # head_dim 128 in 227 KB; beyond that the plan is refused before any
+    # device work
+    st, msg = _create(lib, 1, 1, 1, 6369, 1, 1, 1, 1, 128, 0, 1)
     assert st == 2 and "selection kernel" in msg
     # at the limit validation passes; without a GPU the device query then fails
     h = ctypes.c_void_p()
-    st = lib.bsa_plan_create(ctypes.byref(h), 1, 1, 1, 5856, 1, 1, 1, 1, 128, 0, 1)
+    st = lib.bsa_plan_create(ctypes.byref(h), 1, 1, 1, 6368, 1, 1, 1, 1, 128, 0, 1)
     assert st in (0, 3), lib.bsa_last_error_string().decode()
     if st == 0:
         lib.bsa_plan_destroy(h)
