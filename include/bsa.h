@@ -61,7 +61,7 @@ extern "C" {
 typedef enum {
   BSA_OK = 0,
   BSA_ERR_INVALID_ARG = 1, /* bad shape, pointer, parameter or list width   */
-  BSA_ERR_UNSUPPORTED = 2, /* valid request this build cannot serve          */
+  BSA_ERR_UNSUPPORTED = 2, /* valid request the library does not serve      */
   BSA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed              */
   BSA_ERR_TIMEOUT = 4,     /* a bounded in-kernel wait ran out (dev_status)  */
   BSA_ERR_WORKSPACE = 5,   /* workspace missing or smaller than required     */
