@@ -656,8 +656,11 @@ def run_ours(args, rank, world, local):
         "scheme_generation": dict(scheme, share_of_attn=round(scheme["ms"] / phase_ms["attention"], 4),
                                   frac=round(scheme["achieved_gbs"] / hbm_gbs, 4),
                                   peak_gbs=hbm_gbs, bound="hbm"),
-        # tensor-core plans: centroids, select, 3 pairing kernels, attention
-        "gpu_launches": (6 if plan.info.attn_path == 1 else 4) * args.steps,
+        # per bsa_forward step, tensor-core plans: centroids, select, 4 pairing
+        # kernels (bit sets, candidates, matching, lists; none beyond 1536 video
+        # blocks), attention; other plans: permute, select, attention, unpermute
+        "gpu_launches": ((3 + (4 if plan.info.nb <= 1536 else 0)) if plan.info.attn_path == 1
+                         else 4) * args.steps,
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
