@@ -32,6 +32,8 @@ SMALL = {
     "k_is_one": custom_workload("k_is_one", 1, 8, 16, 16, 2, 4, 16, 2, 128, 0, "bf16", 0, 0.001),
     "topp_tau1": custom_workload("topp_tau1", 1, 8, 16, 16, 2, 4, 16, 2, 128, 0, "bf16", 1, 1.0),
     "single_token": custom_workload("single_token", 1, 1, 1, 1, 1, 8, 16, 1, 128, 0, "bf16", 0, 1.0),
+    # head_dim 64 with text tokens and a ragged grid on the tensor-core path
+    "d64_text": custom_workload("d64_text", 1, 5, 12, 20, 1, 8, 16, 3, 64, 200, "bf16", 0, 0.35),
 }
 
 
