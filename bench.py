@@ -717,48 +717,68 @@ def workload_config(w):
     }
 
 
+class OracleSampler:
+    """The fp64 oracle, as it stands, on bounded samples of a workload: the
+    selection of the whole workload once, then attention on whole random query
+    blocks (all heads) for a time budget per sample."""
+
+    def __init__(self, w, q, k, v):
+        import oracle as orc
+        self.orc, self.w = orc, w
+        self.g = orc.Geometry(*w.geometry_args())
+        self.qn, self.kn, self.vn = (t.float().numpy() for t in (q, k, v))
+        t0 = time.perf_counter()
+        p = orc.scores(self.g, orc.centroids(self.g, self.qn), orc.centroids(self.g, self.kn))
+        self.idx, self.cnt, _ = orc.select(self.g, p, w.mode, w.params)
+        self.t_sel = time.perf_counter() - t0
+        self.full_flop = 4.0 * orc.selected_pairs(self.g, self.idx, self.cnt) * self.g.D
+        self.rng = np.random.default_rng(0)
+        self.valid_tab = {}
+
+    def sample(self, budget_s, chunk=None):
+        """Effective FLOP and seconds of oracle attention over random query
+        blocks (all heads; `chunk` rows of each if given), at least one block.
+        Whole blocks keep the oracle's threads as busy as a full run would."""
+        g = self.g
+        pairs, t_att, nblk = 0, 0.0, 0
+        while True:
+            j = int(self.rng.integers(g.nb))
+            tb, yb, xb = j // (g.nby * g.nbx), (j // g.nbx) % g.nby, j % g.nbx
+            rows = [(t * g.H + y) * g.W + x
+                    for t in range(tb * g.bf, min(g.T, (tb + 1) * g.bf))
+                    for y in range(yb * g.br, min(g.H, (yb + 1) * g.br))
+                    for x in range(xb * g.bc, min(g.W, (xb + 1) * g.bc))]
+            if chunk is not None:
+                c0 = int(self.rng.integers(max(1, len(rows) - chunk + 1)))
+                rows = rows[c0:c0 + chunk]
+            t1 = time.perf_counter()
+            self.orc.attention(g, self.qn, self.kn, self.vn, self.idx, self.cnt, rows=np.array(rows))
+            t_att += time.perf_counter() - t1
+            nblk += 1
+            for b in range(g.B):
+                for h in range(g.Hd):
+                    keys = 0
+                    for jj in self.idx[b, h, j, :self.cnt[b, h, j]]:
+                        if jj not in self.valid_tab:
+                            self.valid_tab[jj] = _valid_count(g, int(jj))
+                        keys += self.valid_tab[jj]
+                    pairs += keys * len(rows)
+            if t_att >= budget_s:
+                return 4.0 * pairs * g.D, t_att, nblk
+
+    def baseline(self, flop, t_att, nblk):
+        return {"value": flop / t_att / 1e12, "unit": "TFLOP/s", "cores": self.orc.threads(),
+                "kind": "oracle", "full_step_flop": self.full_flop,
+                "sample": f"oracle centroids+scores+selection on the full workload "
+                          f"({self.t_sel:.1f} s, once), attention on {nblk} random query blocks "
+                          f"x all {self.g.Hd} heads ({t_att:.1f} s); value = effective FLOP of "
+                          f"the sampled attention / its time"}
+
+
 def cpu_baseline(w, q, k, v, budget_s=20.0):
     """The fp64 oracle, as it stands, on a bounded sample of the workload."""
-    import oracle as orc
-    g = orc.Geometry(*w.geometry_args())
-    qn, kn, vn = (t.float().numpy() for t in (q, k, v))
-    t0 = time.perf_counter()
-    p = orc.scores(g, orc.centroids(g, qn), orc.centroids(g, kn))
-    idx, cnt, _ = orc.select(g, p, w.mode, w.params)
-    t_sel = time.perf_counter() - t0
-    # attention on whole query blocks (all heads), as many as fit the budget
-    rng = np.random.default_rng(0)
-    order = rng.permutation(g.nb)
-    done_rows, pairs, t_att, nblk = [], 0, 0.0, 0
-    valid_tab = {}
-    for j in order:
-        tb, yb, xb = j // (g.nby * g.nbx), (j // g.nbx) % g.nby, j % g.nbx
-        rows = [(t * g.H + y) * g.W + x
-                for t in range(tb * g.bf, min(g.T, (tb + 1) * g.bf))
-                for y in range(yb * g.br, min(g.H, (yb + 1) * g.br))
-                for x in range(xb * g.bc, min(g.W, (xb + 1) * g.bc))]
-        t1 = time.perf_counter()
-        orc.attention(g, qn, kn, vn, idx, cnt, rows=np.array(rows))
-        t_att += time.perf_counter() - t1
-        nblk += 1
-        for b in range(g.B):
-            for h in range(g.Hd):
-                keys = 0
-                for jj in idx[b, h, j, :cnt[b, h, j]]:
-                    if jj not in valid_tab:
-                        valid_tab[jj] = _valid_count(g, int(jj))
-                    keys += valid_tab[jj]
-                pairs += keys * len(rows)
-        if t_att + t_sel >= budget_s:
-            break
-    flops = 4.0 * pairs * g.D
-    tf = flops / t_att / 1e12
-    full_flop = 4.0 * orc.selected_pairs(g, idx, cnt) * g.D
-    return {"value": tf, "unit": "TFLOP/s", "cores": orc.threads(), "kind": "oracle",
-            "full_step_flop": full_flop,
-            "sample": f"oracle centroids+scores+selection on the full workload ({t_sel:.1f} s), "
-                      f"attention on {nblk} random query blocks x all {g.Hd} heads "
-                      f"({t_att:.1f} s); value = effective FLOP of the sampled attention / its time"}
+    o = OracleSampler(w, q, k, v)
+    return o.baseline(*o.sample(max(0.0, budget_s - o.t_sel)))
 
 
 def _valid_count(g, j):
@@ -773,14 +793,19 @@ def run_reference(args, rank, world):
         return
     w = synthetic.workload(args.workload)
     q, k, v = synthetic.make_qkv(w)
-    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
-    vals = []
-    for s in range(args.warmup + args.steps):
-        cb = cpu_baseline(w, q, k, v, budget_s=per_step)
-        if s >= args.warmup:
-            vals.append(cb["value"])
-    value = float(np.mean(vals))
-    cb["value"] = value
+    o = OracleSampler(w, q, k, v)
+    # every step a bounded sample (at least one query block, all heads): about
+    # a minute of oracle attention in all, or one block per step when steps
+    # are many (about 0.7 s each on 16 host cores for the HunyuanVideo shape)
+    per_step = 60.0 / max(1, args.steps + args.warmup)
+    flop = t_att = 0.0
+    nblk = 0
+    for s_i in range(args.warmup + args.steps):
+        f, t, n = o.sample(per_step)
+        if s_i >= args.warmup:
+            flop, t_att, nblk = flop + f, t_att + t, nblk + n
+    cb = o.baseline(flop, t_att, nblk)
+    value = cb["value"]
     # one whole step of the workload at the sampled rate
     ms_full = cb["full_step_flop"] / (value * 1e12) * 1e3
     config = workload_config(w)
