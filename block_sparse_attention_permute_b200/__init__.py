@@ -76,6 +76,7 @@ def load():
         "bsa_attention": [P, P, P, P, P, P, I, P, P, P],
         "bsa_forward": [P, P, P, P, I, P, I, P, P, P, P, Z, P, P],
         "bsa_check_status": [P, P],
+        "bsa_plan_set_watchdog": [P, ctypes.c_longlong, I],
         "bsa_sics": [P, P, P, P],
         "bsa_kmax_for_union": [P, I, P, P, ctypes.POINTER(I)],
         "bsa_union_workspace_size": [P, I, P, ctypes.POINTER(Z), ctypes.POINTER(Z)],
@@ -444,6 +445,11 @@ class Plan:
     def check_status(self):
         """Synchronise the current stream and raise if a kernel recorded an error."""
         _check(load().bsa_check_status(self._h, _stream(self.device)))
+
+    def set_watchdog(self, wait_limit_cycles=0, withhold_copy=0):
+        """Bound of the attention kernel's in-kernel waits (0 = default, about a
+        second) and the timeout path's test hook (bsa_plan_set_watchdog)."""
+        _check(load().bsa_plan_set_watchdog(self._h, int(wait_limit_cycles), int(withhold_copy)))
 
 
 def aggregation_scores(plans, x):

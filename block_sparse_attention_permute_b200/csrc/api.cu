@@ -17,6 +17,8 @@ struct bsa_plan_s {
   int device;
   int attn_path;        // 1 tcgen05, 0 SIMT
   int32_t* d_status;    // device status word
+  long long wait_limit; // bound of the attention kernel's waits, SM cycles (0 = default)
+  int hold_load;        // test hook of the timeout path (0 = off)
   uint32_t* d_masks;    // [(nb + nb_text) * 4] slot validity bits (bs == 128)
 };
 
@@ -273,6 +275,8 @@ bsa_status run_attention(const bsa_plan_s* p, const void* q, const void* k, cons
   a.q = q; a.k = k; a.v = v; a.o = o; a.idx = idx; a.cnt = cnt; a.masks = p->d_masks;
   a.status = dev_status ? dev_status : p->d_status;
   a.kmax = kmax;
+  a.wait_limit = p->wait_limit;
+  a.hold_load = p->hold_load;
   a.scale = (float)(1.0 / std::sqrt((double)p->g.D));
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->g.D));
   cudaError_t e;
@@ -391,7 +395,6 @@ bsa_status run_attention_orig(const bsa_plan_s* p, const void* q, const void* k,
     if ((s = make_orig_maps(&maps.v, &maps.vt, vb, p->g)) != BSA_OK) return s;
     bsa::AttnArgs a;
     std::memset(&a, 0, sizeof(a));
-  std::memset(&a, 0, sizeof(a));
     a.q = qb; a.k = kb; a.v = vb;
     a.o = reinterpret_cast<char*>(o) + b * per_batch;
     a.idx = idx + (size_t)b * p->g.Hd * p->g.nb * kmax;
@@ -399,6 +402,8 @@ bsa_status run_attention_orig(const bsa_plan_s* p, const void* q, const void* k,
     a.masks = p->d_masks;
     a.status = dev_status ? dev_status : p->d_status;
     a.kmax = kmax;
+    a.wait_limit = p->wait_limit;
+    a.hold_load = p->hold_load;
     a.scale = (float)(1.0 / std::sqrt((double)p->g.D));
     a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->g.D));
     a.map = hm;
@@ -615,6 +620,8 @@ bsa_status bsa_plan_create(bsa_plan_t* out, int batch, int T, int H, int W, int 
   p.attn_path = (dtype == BSA_BF16 && bs == 128) ? 1 : 0;
   p.d_status = nullptr;
   p.d_masks = nullptr;
+  p.wait_limit = 0;
+  p.hold_load = 0;
 
   cudaError_t e = cudaGetDevice(&p.device);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -1083,6 +1090,15 @@ bsa_status bsa_check_status(bsa_plan_t p, void* stream) {
   if (v == 0) return BSA_OK;
   return fail((bsa_status)v, "kernel reported status %d (%s)", v,
               v == BSA_ERR_TIMEOUT ? "a bounded wait ran out" : "an index list entry was out of range");
+}
+
+bsa_status bsa_plan_set_watchdog(bsa_plan_t p, long long wait_limit_cycles, int withhold_copy) {
+  if (p == nullptr) return fail(BSA_ERR_INVALID_ARG, "plan is NULL");
+  if (wait_limit_cycles < 0 || withhold_copy < 0)
+    return fail(BSA_ERR_INVALID_ARG, "wait limit and withheld copy must be >= 0");
+  p->wait_limit = wait_limit_cycles;
+  p->hold_load = withhold_copy;
+  return BSA_OK;
 }
 
 }  // extern "C"

@@ -221,7 +221,6 @@ constexpr int kTcThreads = 384;
 constexpr int kRegsLaunch = 168, kRegsSoftmax = 216, kRegsSmall = 72;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsSmall <= kTcThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
-constexpr int kExpFmaPairsPer8 = 0;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;      // log2 units
 
@@ -288,6 +287,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t bar0 = sb + L::kBars;
   auto bar = [&](int x) { return bar0 + 8u * (uint32_t)x; };
   volatile int* abort = reinterpret_cast<volatile int*>(sm + L::kAbort);
+  const long long lim = a.wait_limit > 0 ? a.wait_limit : kWaitLimitDefault;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nbk = g.nb + g.nb_text;
@@ -380,9 +380,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (x == 1 && s < c_shared) return true;
         int j = block_at(x, s);
         if (j < 0) { bad = true; j = 0; }   // load some tile; the softmax masks the step
+        // test hook: a copy that never lands, so that the consumer's wait runs out
+        if (pos + 1 == a.hold_load && blockIdx.x == 0) return false;
         const int slot = pos % L::kStages;
         if (pos >= L::kStages &&
-            !mbar_wait(bar(L::kBarEmpty + slot), ((pos / L::kStages) - 1) & 1, abort))
+            !mbar_wait(bar(L::kBarEmpty + slot), ((pos / L::kStages) - 1) & 1, abort, lim))
           return false;
         const uint32_t dst = sRing + slot * kTileBytes;
         mbar_arrive_expect_tx(bar(L::kBarFull + slot), kTileBytes);
@@ -391,18 +393,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         return true;
       });
       if (bad) set_status(a.status, 6);
-      // Never leave the CTA with a copy in flight: wait for the last loads.
+      // Never leave the CTA with a copy in flight: wait for the Q tiles and
+      // the last kStages K/V copies issued (each slot's latest copy), also
+      // after an abort (these waits ignore it; issued copies always land).
       for (int x = 0; x < 2; ++x)
-        if ((x ? n1 : n0) > 0) mbar_wait(bar(L::kBarQ + x), 0, abort);
+        if ((x ? n1 : n0) > 0) mbar_wait_drain(bar(L::kBarQ + x), 0, lim);
       for (int p = (pos > L::kStages ? pos - L::kStages : 0); p < pos; ++p)
-        mbar_wait(bar(L::kBarFull + p % L::kStages), (p / L::kStages) & 1, abort);
+        mbar_wait_drain(bar(L::kBarFull + p % L::kStages), (p / L::kStages) & 1, lim);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = true;
       for (int x = 0; x < 2; ++x)
-        if ((x ? n1 : n0) > 0 && !mbar_wait(bar(L::kBarQ + x), 0, abort)) ok = false;
+        if ((x ? n1 : n0) > 0 && !mbar_wait(bar(L::kBarQ + x), 0, abort, lim)) ok = false;
       tc_fence_after();
       int pos = 0;
       int shared_slot[2] = {0, 0};   // ring slot of tile 0's K (S) and V (PV) of a shared step
@@ -416,7 +420,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             slot = kind == 0 ? shared_slot[0] : shared_slot[1];
           } else {
             slot = pos % L::kStages;
-            if (!mbar_wait(bar(L::kBarFull + slot), (pos / L::kStages) & 1, abort)) return false;
+            if (!mbar_wait(bar(L::kBarFull + slot), (pos / L::kStages) & 1, abort, lim)) return false;
             tc_fence_after();
             ++pos;
             if (shared) {
@@ -436,7 +440,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             tc_commit(bar(L::kBarS + x));
           } else {
-            if (!mbar_wait(bar(L::kBarP + x), s & 1, abort)) return false;
+            if (!mbar_wait(bar(L::kBarP + x), s & 1, abort, lim)) return false;
             tc_fence_after();
             const uint32_t tO = tmem + 256u + 128u * x;
 #pragma unroll
@@ -449,9 +453,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           return true;
         });
       }
-      // Every MMA issued must be complete before TMEM is released.
+      // Every MMA issued must be complete before TMEM is released, also
+      // after an abort (the commit tracks all of them; the wait ignores abort).
       tc_commit(bar(L::kBarFinal));
-      mbar_wait(bar(L::kBarFinal), 0, abort);
+      mbar_wait_drain(bar(L::kBarFinal), 0, lim);
     }
    }
   } else {
@@ -481,7 +486,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           mw_next = j_next >= 0 ? __ldg(reinterpret_cast<const uint4*>(a.masks) + j_next)
                                 : make_uint4(0u, 0u, 0u, 0u);
         }
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + x), s & 1, abort))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + x), s & 1, abort, lim))) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[128];
         TMEM_LD32(tS + 0, (sr + 0));
@@ -526,9 +531,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int c = 0; c < 64; ++c) {
           const float2 t = fma2(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])),
                                 sl2, neg_m);
-          // kExpFmaPairsPer8 of every 8 pairs take the FMA-pipe exponential.
-          const float2 p = ((c & 7) < kExpFmaPairsPer8) ? exp2_fma2(t)
-                                                        : make_float2(fast_ex2(t.x), fast_ex2(t.y));
+          const float2 p = make_float2(fast_ex2(t.x), fast_ex2(t.y));
           acc[c & 3] = add2(acc[c & 3], p);
           pk[c] = pack_bf16x2(p.x, p.y);
         }
@@ -556,7 +559,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       // ---- epilogue: O / l -> blocked output row
       if (ok && n > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarO + x), 0, abort));
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarO + x), 0, abort, lim));
         tc_fence_after();
       }
       const uint4 qm = __ldg(reinterpret_cast<const uint4*>(a.masks) + qi);

@@ -99,20 +99,37 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity
   return ok != 0;
 }
 
+// Default bound of an in-kernel wait, in SM clock cycles (about a second).
+constexpr long long kWaitLimitDefault = 1ll << 31;
+
 // Bounded wait: parks on try_wait (1 ms suspend hint per attempt) until the
-// phase with `parity` completes, another role raised *abort, or ~2^31 cycles
-// (about a second) have passed; in the last case it raises *abort itself.
-// Returns true on completion.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+// phase with `parity` completes, another role raised *abort, or `limit`
+// cycles have passed; in the last case it raises *abort itself.  Returns
+// true on completion.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (true) {
     if (mbar_try_wait_hint(bar, parity, 1000000u)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > (1ll << 31)) {
+    if (clock64() - t0 > limit) {
       *abort = 1;
       return false;
     }
+  }
+}
+
+// Wait used after an abort to collect work this CTA has already issued (TMA
+// copies, MMAs), which completes whatever the other roles do: it ignores the
+// abort flag and gives up only after `limit` cycles.  Returns true on
+// completion.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, long long limit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait_hint(bar, parity, 1000000u)) return true;
+    if (clock64() - t0 > limit) return false;
   }
 }
 
@@ -300,27 +317,6 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
       : "=l"(reinterpret_cast<uint64_t&>(d))
       : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)));
   return d;
-}
-
-// 2^x for two arguments on the FMA pipe (relieves the MUFU unit, which runs at
-// a quarter of the FMA rate).  Cody-Waite style split x = j + f with
-// j = rint(x) taken by the 1.5*2^23 magic-number addition and f in [-1/2, 1/2];
-// 2^f from a cubic fitted in this repository for minimum relative error on
-// that interval (7.5e-5, far below the bf16 rounding of the result's use);
-// j is added to the exponent field.  Arguments below -125, -inf included,
-// give exactly 0.
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-  const float2 xc = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
-  const float2 t = add2(xc, make_float2(12582912.f, 12582912.f));
-  const float2 j = add2(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = fma2(j, make_float2(-1.f, -1.f), xc);
-  float2 p = fma2(make_float2(0.05517124757170677f, 0.05517124757170677f), f,
-                  make_float2(0.24261054396629333f, 0.24261054396629333f));
-  p = fma2(p, f, make_float2(0.6932610273361206f, 0.6932610273361206f));
-  p = fma2(p, f, make_float2(0.9999281167984009f, 0.9999281167984009f));
-  const uint32_t bx = __float_as_uint(p.x) + (__float_as_uint(t.x) << 23);
-  const uint32_t by = __float_as_uint(p.y) + (__float_as_uint(t.y) << 23);
-  return make_float2(x.x < -125.f ? 0.f : __uint_as_float(bx), x.y < -125.f ? 0.f : __uint_as_float(by));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -80,6 +80,8 @@ struct AttnArgs {
   const uint32_t* masks;  // [(nb + nb_text) * 4] slot validity bits (bs == 128 only)
   int32_t* status;        // device status word
   int kmax;
+  long long wait_limit;   // bound of every in-kernel wait, SM cycles (0 = kWaitLimitDefault)
+  int hold_load;          // test hook: n > 0 = CTA 0 never issues its n-th K/V copy; 0 = off
   float scale;            // 1/sqrt(D)
   float scale_log2;       // log2(e)/sqrt(D)
   HeadMap map;

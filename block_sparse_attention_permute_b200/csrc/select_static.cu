@@ -11,7 +11,9 @@
 //
 // Set-up: the first call on each device looks up that device's copy of the
 // array with cudaGetSymbolAddress (with that device current) and caches the
-// address; make that first call before any stream capture begins.
+// address together with the id of the current context; a later call in
+// another context (after a device reset, say) looks it up again.  Make the
+// first call on a device before any stream capture begins.
 // Sharing: all calls on a device use the same array and it keeps the last
 // call's contents.  Every centroid is rewritten by each call before it is
 // read, so nothing needs clearing, but calls whose kernels overlap on the
@@ -32,17 +34,52 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
+unsigned long long g_scratch_ctx[kMaxDevices] = {0};   // context the address belongs to
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current CUDA context (0 if the driver
+// cannot tell): a device reset or a re-created primary context gets a new id,
+// and with it a new copy of the array at a new address.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+        qb == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(b);
+    looked_up = true;
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS ||
+      ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 // Device address of this device's copy of g_select_scratch (the host-side
-// name is only a stand-in and must never be handed to a kernel).
+// name is only a stand-in and must never be handed to a kernel).  Looked up
+// once per device and context; looked up again whenever the current context
+// differs from the one the cached address came from (or cannot be told).
 cudaError_t scratch_for_device(int dev, void** out) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (g_scratch_ptr[dev] == nullptr || ctx == 0 || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_select_scratch);
     if (e != cudaSuccess) return e;
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;

@@ -224,8 +224,10 @@ bsa_status bsa_select_centroids(bsa_plan_t plan, const float* q_cent,
  *   to 256 bytes) must fit in 16 MiB, else BSA_ERR_UNSUPPORTED and nothing is
  *   launched.
  *   The first call on a device looks up that device's copy of the array
- *   (cudaGetSymbolAddress, with the device current) and caches it; make that
- *   first call before any stream capture begins.
+ *   (cudaGetSymbolAddress, with the device current) and caches it with the
+ *   id of the current context (a call in another context, e.g. after a
+ *   device reset, looks it up again); make that first call before any stream
+ *   capture begins.
  *   All calls on a device share the array and it keeps the last call's
  *   contents (each call rewrites every centroid it reads, so nothing needs
  *   clearing); calls whose kernels overlap on the GPU race on it. */
@@ -490,6 +492,27 @@ bsa_status bsa_attention_paired(bsa_plan_t plan, const void* q, const void* k,
 /* bsa_check_status — synchronise `stream`, read and clear the plan-owned
  * status word; returns BSA_OK or the recorded error. */
 bsa_status bsa_check_status(bsa_plan_t plan, void* stream);
+
+/* bsa_plan_set_watchdog — bound of the tensor-core attention kernel's
+ * in-kernel waits (failure detection; no counterpart on the pages, which
+ * describe no failure handling).
+ *   wait_limit_cycles  every mbarrier wait of the kernel (a K/V copy landing,
+ *                      S or P ready, a ring slot freed) gives up after this
+ *                      many SM clock cycles; 0 = the default of 2^31 (about
+ *                      a second).  When a wait runs out the kernel raises a
+ *                      CTA-wide abort, waits (with the same bound) for the
+ *                      copies and MMAs it has already issued, frees its TMEM,
+ *                      writes zeros for its rows and records BSA_ERR_TIMEOUT
+ *                      in the status word; the context stays usable.
+ *   withhold_copy      test hook of that path: n > 0 makes CTA 0 of every
+ *                      tensor-core attention launch skip its n-th K/V copy
+ *                      (so its consumer's wait runs out); 0 = off.  Never set
+ *                      it outside tests.
+ * Takes effect for launches issued after the call; do not change it while a
+ * call on this plan is being issued on another thread.  Negative values are
+ * BSA_ERR_INVALID_ARG. */
+bsa_status bsa_plan_set_watchdog(bsa_plan_t plan, long long wait_limit_cycles,
+                                 int withhold_copy);
 
 /* Thread-local message describing the last non-OK return of this thread. */
 const char* bsa_last_error_string(void);
