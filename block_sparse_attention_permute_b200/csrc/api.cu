@@ -277,6 +277,9 @@ bsa_status run_attention(const bsa_plan_s* p, const void* q, const void* k, cons
   a.kmax = kmax;
   a.wait_limit = p->wait_limit;
   a.hold_load = p->hold_load;
+  a.div_nbx = make_fastdiv((uint32_t)p->g.nbx);
+  a.div_nby = make_fastdiv((uint32_t)p->g.nby);
+  a.div_hd = make_fastdiv((uint32_t)p->g.Hd);
   a.scale = (float)(1.0 / std::sqrt((double)p->g.D));
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->g.D));
   cudaError_t e;
@@ -404,6 +407,9 @@ bsa_status run_attention_orig(const bsa_plan_s* p, const void* q, const void* k,
     a.kmax = kmax;
     a.wait_limit = p->wait_limit;
     a.hold_load = p->hold_load;
+    a.div_nbx = make_fastdiv((uint32_t)p->g.nbx);
+    a.div_nby = make_fastdiv((uint32_t)p->g.nby);
+    a.div_hd = make_fastdiv((uint32_t)p->g.Hd);
     a.scale = (float)(1.0 / std::sqrt((double)p->g.D));
     a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->g.D));
     a.map = hm;

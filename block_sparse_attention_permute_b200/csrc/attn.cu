@@ -252,8 +252,9 @@ __device__ __forceinline__ bool for_each_event(int n0, int n1, F&& f) {
 // (dt, dy, dx) and whose out-of-range part (the grid's padding) is zero-filled,
 // or a 3D box (d, head, token) over the text tokens.
 template <bool ORIG, int HD>
-__device__ __forceinline__ void load_tile(const TileMaps& m, int which, const Geo& g, long long bh,
-                                          int j, uint32_t dst, uint32_t bar) {
+__device__ __forceinline__ void load_tile(const TileMaps& m, int which, const Geo& g,
+                                          const AttnArgs& a, long long bh, int j, uint32_t dst,
+                                          uint32_t bar) {
   constexpr int kPanel = 128 * 128;
   if (!ORIG) {
     const int row = (int)((bh * (g.nb + g.nb_text) + j) * 128);
@@ -261,9 +262,11 @@ __device__ __forceinline__ void load_tile(const TileMaps& m, int which, const Ge
 #pragma unroll
     for (int p = 0; p < HD / 64; ++p) tma_load_2d(dst + p * kPanel, map, 64 * p, row, bar);
   } else {
-    const int h = (int)(bh % g.Hd);
+    // one batch element per launch: bh < Hd, so h = bh (kept general)
+    const int h = (int)bh - (int)fdiv((uint32_t)bh, a.div_hd) * g.Hd;
     if (j < g.nb) {
-      const int xb = j % g.nbx, yb = (j / g.nbx) % g.nby, tb = j / (g.nbx * g.nby);
+      const int q1 = (int)fdiv((uint32_t)j, a.div_nbx), tb = (int)fdiv((uint32_t)q1, a.div_nby);
+      const int xb = j - q1 * g.nbx, yb = q1 - tb * g.nby;
       const CUtensorMap* map = which == 0 ? &m.q : (which == 1 ? &m.k : &m.v);
 #pragma unroll
       for (int p = 0; p < HD / 64; ++p)
@@ -370,7 +373,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int x = 0; x < 2; ++x) {
         if ((x ? n1 : n0) == 0) continue;
         mbar_arrive_expect_tx(bar(L::kBarQ + x), kTileBytes);
-        load_tile<ORIG, HD>(maps, 0, g, x ? bh1 : bh0, x ? i1 : i0, sb + L::kQ + x * kTileBytes,
+        load_tile<ORIG, HD>(maps, 0, g, a, x ? bh1 : bh0, x ? i1 : i0, sb + L::kQ + x * kTileBytes,
                             bar(L::kBarQ + x));
       }
       int pos = 0;
@@ -388,7 +391,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           return false;
         const uint32_t dst = sRing + slot * kTileBytes;
         mbar_arrive_expect_tx(bar(L::kBarFull + slot), kTileBytes);
-        load_tile<ORIG, HD>(maps, kind == 0 ? 1 : 2, g, x ? bh1 : bh0, j, dst, bar(L::kBarFull + slot));
+        load_tile<ORIG, HD>(maps, kind == 0 ? 1 : 2, g, a, x ? bh1 : bh0, j, dst, bar(L::kBarFull + slot));
         ++pos;
         return true;
       });

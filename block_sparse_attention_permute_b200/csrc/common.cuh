@@ -42,6 +42,33 @@ __host__ __device__ __forceinline__ int block_valid_count(const Geo& g, int j) {
   return (int)(rem < g.bs ? rem : g.bs);
 }
 
+// Division of a non-negative 32-bit integer by a run-time invariant divisor
+// d >= 1 with a multiply-high and a shift (Granlund and Montgomery,
+// "Division by Invariant Integers using Multiplication", 1994, Fig. 4.1):
+// l = ceil(log2 d), m = floor(2^32 (2^l - d) / d) + 1, n / d =
+// (mulhi(m, n) + n) >> l.  On the GPU a division by a register value goes
+// through the MUFU reciprocal unit, which the softmax keeps saturated with
+// exponentials; this form uses the integer pipe only.
+struct FastDiv {
+  uint32_t m, l, d;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  f.l = 0;
+  while ((1ull << f.l) < d) ++f.l;
+  f.m = (uint32_t)(((1ull << 32) * ((1ull << f.l) - d)) / d + 1);
+  return f;
+}
+__host__ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+#if defined(__CUDA_ARCH__)
+  const uint32_t hi = __umulhi(f.m, n);
+#else
+  const uint32_t hi = (uint32_t)(((uint64_t)f.m * n) >> 32);
+#endif
+  return (uint32_t)(((uint64_t)hi + n) >> f.l);
+}
+
 // Maximum number of heads a selection call carries per-head parameters for.
 #define BSA_MAX_HEADS 256
 

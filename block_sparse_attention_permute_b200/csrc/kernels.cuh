@@ -95,6 +95,9 @@ struct AttnArgs {
   const int32_t* pair_sched;
   const int32_t* pair_lists;
   int pairs_per_head, text_pairs;
+  // divisors of the per-copy block coordinates (nbx, nby, Hd), so that the
+  // copy-issuing thread divides without the MUFU unit
+  FastDiv div_nbx, div_nby, div_hd;
 };
 
 // Pairing of the query tiles of each (b, h) into CTA pairs that share key
