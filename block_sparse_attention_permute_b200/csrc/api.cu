@@ -19,6 +19,7 @@ struct bsa_plan_s {
   int32_t* d_status;    // device status word
   long long wait_limit; // bound of the attention kernel's waits, SM cycles (0 = default)
   int hold_load;        // test hook of the timeout path (0 = off)
+  int sm_count;         // multiprocessors of the plan's device
   uint32_t* d_masks;    // [(nb + nb_text) * 4] slot validity bits (bs == 128)
 };
 
@@ -327,6 +328,17 @@ bsa_status run_centroids(const bsa_plan_s* p, const void* q, const void* k, floa
 // Query tiles per head paired for K/V sharing (pair.cu): text pairs, then
 // video pairs.
 int text_pairs(const Geo& g) { return (g.nb_text + 1) / 2; }
+// How many head windows one text pair of the paired schedule spans: a text
+// pair is (nb + nb_text) steps of two tiles on one SM, while the whole GPU
+// works through one head's nb * list + text tile-steps in a window; lists are
+// at most kmax long (the bound errs towards placing text pairs late; +1 for
+// margin).
+int text_lead(const Geo& g, int kmax, int sms) {
+  if (g.nb_text == 0) return 1;
+  const double text_work = 2.0 * (g.nb + g.nb_text);
+  const double window = ((double)g.nb * kmax + 2.0 * g.nb_text * (g.nb + g.nb_text)) / (sms > 0 ? sms : 148);
+  return (int)std::ceil(text_work / window) + 1;
+}
 int pairs_per_head(const Geo& g) { return text_pairs(g) + (g.nb + 1) / 2; }
 size_t pairing_bytes(const bsa_plan_s* p, int kmax) {
   const size_t bh = (size_t)p->g.B * p->g.Hd, pph = pairs_per_head(p->g);
@@ -419,6 +431,7 @@ bsa_status run_attention_orig(const bsa_plan_s* p, const void* q, const void* k,
       a.pair_lists = pair_lists + (long long)b * p->g.Hd * pph * 2 * kmax;
       a.pairs_per_head = (int)pph;
       a.text_pairs = text_pairs(p->g);
+      a.text_lead = text_lead(p->g, kmax, p->sm_count);
     }
     cudaError_t e = bsa::launch_attn_tc_orig(g1, a, maps, st);
     if (e != cudaSuccess) return cuda_fail(e, "attention kernel");
@@ -631,6 +644,9 @@ bsa_status bsa_plan_create(bsa_plan_t* out, int batch, int T, int H, int W, int 
 
   cudaError_t e = cudaGetDevice(&p.device);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  p.sm_count = 148;
+  if ((e = cudaDeviceGetAttribute(&p.sm_count, cudaDevAttrMultiProcessorCount, p.device)) != cudaSuccess)
+    return cuda_fail(e, "cudaDeviceGetAttribute");
   const int nbk = g.nb + g.nb_text;
   std::vector<uint32_t> masks((size_t)nbk * 4, 0u);
   if (bs <= 128)

@@ -319,14 +319,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // the video pairs; entry (h, t) names the two tiles and the shared count.
     const int n_heads = map_count(a.map, g.B * g.Hd);
     const int vpairs = a.pairs_per_head - a.text_pairs;
+    // Head-major order, each head's text pairs placed at the start of its own
+    // window so that they read its K / V while its video pairs do (one pass
+    // over the head's K / V from DRAM).  A text pair runs about text_lead
+    // head windows, so the text pairs of the last text_lead heads are issued
+    // together at the start of head n_heads - text_lead's window, early
+    // enough to finish with the rest of the launch.
+    const int tp = a.text_pairs, per = tp + vpairs;
+    const int lead = min(max(a.text_lead, 1), n_heads);
+    const int h_split = n_heads - lead;            // heads 0 .. h_split-1: own group
     int e = blockIdx.x, m, t;
-    if (e < n_heads * a.text_pairs) {
-      m = e / a.text_pairs;
-      t = e % a.text_pairs;
+    if (e < h_split * per) {
+      m = e / per;
+      t = e % per;
     } else {
-      e -= n_heads * a.text_pairs;
-      m = e / vpairs;
-      t = a.text_pairs + e % vpairs;
+      e -= h_split * per;
+      if (e < lead * tp) {
+        m = h_split + e / tp;
+        t = e % tp;
+      } else {
+        e -= lead * tp;
+        m = h_split + e / vpairs;
+        t = tp + e % vpairs;
+      }
     }
     const long long bh = map_bh(a.map, m);
     const long long ent = bh * a.pairs_per_head + t;

@@ -95,6 +95,7 @@ struct AttnArgs {
   const int32_t* pair_sched;
   const int32_t* pair_lists;
   int pairs_per_head, text_pairs;
+  int text_lead;          // head windows a text pair spans (its position in the order)
   // divisors of the per-copy block coordinates (nbx, nby, Hd), so that the
   // copy-issuing thread divides without the MUFU unit
   FastDiv div_nbx, div_nby, div_hd;
