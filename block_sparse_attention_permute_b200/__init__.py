@@ -77,6 +77,7 @@ def load():
         "bsa_forward": [P, P, P, P, I, P, I, P, P, P, P, Z, P, P],
         "bsa_check_status": [P, P],
         "bsa_plan_set_watchdog": [P, ctypes.c_longlong, I],
+        "bsa_forward_timed": [P, P, P, P, I, P, I, P, P, P, P, Z, P, P, ctypes.POINTER(Timings)],
         "bsa_sics": [P, P, P, P],
         "bsa_kmax_for_union": [P, I, P, P, ctypes.POINTER(I)],
         "bsa_union_workspace_size": [P, I, P, ctypes.POINTER(Z), ctypes.POINTER(Z)],
@@ -121,6 +122,15 @@ def _params(p, heads):
     if len(p) != heads:
         raise BsaError(1, f"expected {heads} per-head parameters, got {len(p)}")
     return arr
+
+
+class Timings(ctypes.Structure):
+    """bsa_timings_t: device milliseconds of the phases of one bsa_forward call."""
+    _fields_ = [(n, ctypes.c_float) for n in ("summaries_ms", "select_ms", "pairing_ms",
+                                               "attention_ms", "unpermute_ms", "total_ms")]
+
+    def as_dict(self):
+        return {n: float(getattr(self, n)) for n, _ in self._fields_}
 
 
 class MaskUnion(ctypes.Structure):
@@ -339,6 +349,22 @@ class Plan:
                                   _params(params, self.info.heads), kmax, _ptr(out), _ptr(idx),
                                   _ptr(cnt), _ptr(ws), ws.numel(), None, _stream(self.device)))
         return (out, idx, cnt) if return_lists else out
+
+    def forward_timed(self, q, k, v, mode, params, kmax=None, out=None, workspace=None):
+        """bsa_forward_timed: the forward plus the device time of each phase
+        (synchronises); returns (out, dict of milliseconds)."""
+        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+            self._check_tensor(t, self.orig_shape, name=n)
+        kmax = self.kmax_for(mode, params) if kmax is None else kmax
+        out = self._new(self.orig_shape) if out is None else out
+        need = self.workspace_size(kmax)[1]
+        ws = self._new((need,), torch.uint8) if workspace is None else workspace
+        t = Timings()
+        _check(load().bsa_forward_timed(self._h, _ptr(q), _ptr(k), _ptr(v), mode,
+                                        _params(params, self.info.heads), kmax, _ptr(out), None,
+                                        None, _ptr(ws), ws.numel(), None, _stream(self.device),
+                                        ctypes.byref(t)))
+        return out, t.as_dict()
 
     # --------------------------------------------------------- mask union
     def kmax_for_union(self, mode, params, union) -> int:

@@ -155,6 +155,20 @@ bsa_status make_orig_maps(CUtensorMap* video, CUtensorMap* text, const void* x, 
   return BSA_OK;
 }
 
+// Events at the phase boundaries of one forward call (bsa_forward_timed):
+// mark() records the next event on the call's stream; a null timer records
+// nothing.
+struct PhaseTimer {
+  cudaEvent_t ev[6];
+  int n = 0;
+  cudaStream_t st = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+void mark(PhaseTimer* t) {
+  if (t == nullptr || t->n >= 6 || t->err != cudaSuccess) return;
+  t->err = cudaEventRecord(t->ev[t->n++], t->st);
+}
+
 // Host copy of a validated mask union (window, sink, intra selection).
 struct UnionOpts {
   int win_left = -1, win_right = -1;
@@ -447,19 +461,25 @@ bsa_status run_forward_fused(const bsa_plan_s* p, const void* q, const void* k, 
                              int32_t* idx, int32_t* cnt, float* qc, float* kc,
                              int32_t* dev_status, cudaStream_t st, const UnionOpts* uo,
                              float* k_sics, uint32_t* bits, int est, char* pair_ws,
-                             const bsa::HeadMap* map = nullptr) {
+                             const bsa::HeadMap* map = nullptr, PhaseTimer* timer = nullptr) {
+  mark(timer);
   bsa_status s = run_centroids(p, q, k, qc, kc, st, k_sics, est != bsa::kEstMean, map);
   if (s != BSA_OK) return s;
+  mark(timer);
   if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st, uo, k_sics, bits, est,
                       map)) != BSA_OK)
     return s;
+  mark(timer);
   int32_t* sched = nullptr;
   int32_t* lists = nullptr;
   // pairing only reorders the work; plans beyond its block limit run unpaired
   if (pair_ws != nullptr && bsa::pairing_supported(p->g) &&
       (s = run_pairing(p, idx, cnt, kmax, pair_ws, &sched, &lists, st, map)) != BSA_OK)
     return s;
-  return run_attention_orig(p, q, k, v, idx, cnt, kmax, o, dev_status, st, map, sched, lists);
+  mark(timer);
+  s = run_attention_orig(p, q, k, v, idx, cnt, kmax, o, dev_status, st, map, sched, lists);
+  mark(timer);
+  return s;
 }
 
 // kmax a list can need under the union: the inter bound plus the blocks the
@@ -492,7 +512,7 @@ bsa_status forward_impl(bsa_plan_t p, const void* q, const void* k, const void* 
                         bsa_select_mode mode, const double* param, const bsa_mask_union_t* u,
                         int kmax, void* o, int32_t* idx_out, int32_t* cnt_out, void* ws,
                         size_t ws_bytes, int32_t* dev_status, void* stream,
-                        int est = bsa::kEstMean) {
+                        int est = bsa::kEstMean, PhaseTimer* timer = nullptr) {
   bsa_status s = check_plan(p);
   if (s != BSA_OK) return s;
   if (est != bsa::kEstMean && est != bsa::kEstDsa && est != bsa::kEstDsa2)
@@ -540,7 +560,7 @@ bsa_status forward_impl(bsa_plan_t p, const void* q, const void* k, const void* 
   const UnionOpts* up = u ? &uo : nullptr;
   if (p->attn_path == 1)
     return run_forward_fused(p, q, k, v, mode, param, kmax, o, idx, cnt, qc, kc, dev_status, st, up,
-                             k_sics, bits, est, w);
+                             k_sics, bits, est, w, nullptr, timer);
   bsa::GatherArgs a;
   std::memset(&a, 0, sizeof(a));
   a.src[0] = q; a.src[1] = k; a.src[2] = v;
@@ -552,12 +572,18 @@ bsa_status forward_impl(bsa_plan_t p, const void* q, const void* k, const void* 
   }
   a.sics[1] = k_sics;
   a.ntensors = 3;
+  mark(timer);
   cudaError_t e = bsa::launch_permute(p->g, p->dtype == BSA_BF16, a, st);
   if (e != cudaSuccess) return cuda_fail(e, "permute kernel");
+  mark(timer);
   if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st, up, k_sics, bits, est)) != BSA_OK)
     return s;
+  mark(timer);
   if ((s = run_attention(p, q_blk, k_blk, v_blk, idx, cnt, kmax, o_blk, dev_status, st)) != BSA_OK) return s;
-  return bsa_unpermute(p, o_blk, o, stream);
+  mark(timer);
+  s = bsa_unpermute(p, o_blk, o, stream);
+  mark(timer);
+  return s;
 }
 
 // Workspace of one scheme group of bsa_forward_grouped: its centroids, its
@@ -819,6 +845,56 @@ bsa_status bsa_forward(bsa_plan_t p, const void* q, const void* k, const void* v
                        int32_t* dev_status, void* stream) {
   return forward_impl(p, q, k, v, mode, param, nullptr, kmax, o, idx_out, cnt_out, ws, ws_bytes,
                       dev_status, stream);
+}
+
+bsa_status bsa_forward_timed(bsa_plan_t p, const void* q, const void* k, const void* v,
+                             bsa_select_mode mode, const double* param, int kmax, void* o,
+                             int32_t* idx_out, int32_t* cnt_out, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, void* stream, bsa_timings_t* timings) {
+  if (timings == nullptr) return fail(BSA_ERR_INVALID_ARG, "timings is NULL");
+  std::memset(timings, 0, sizeof(*timings));
+  PhaseTimer t;
+  t.st = (cudaStream_t)stream;
+  int made = 0;
+  cudaError_t e = cudaSuccess;
+  for (; made < 6 && e == cudaSuccess; ++made) e = cudaEventCreate(&t.ev[made]);
+  if (e != cudaSuccess) made--;
+  auto destroy = [&]() {
+    for (int i = 0; i < made; ++i) cudaEventDestroy(t.ev[i]);
+  };
+  if (e != cudaSuccess) {
+    destroy();
+    return cuda_fail(e, "cudaEventCreate");
+  }
+  bsa_status s = forward_impl(p, q, k, v, mode, param, nullptr, kmax, o, idx_out, cnt_out, ws,
+                              ws_bytes, dev_status, stream, bsa::kEstMean, &t);
+  if (s == BSA_OK && t.err != cudaSuccess) s = cuda_fail(t.err, "cudaEventRecord");
+  if (s == BSA_OK && (e = cudaEventSynchronize(t.ev[t.n - 1])) != cudaSuccess) s = cuda_fail(e, "cudaEventSynchronize");
+  if (s == BSA_OK) {
+    float ms[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i + 1 < t.n && s == BSA_OK; ++i)
+      if ((e = cudaEventElapsedTime(&ms[i], t.ev[i], t.ev[i + 1])) != cudaSuccess)
+        s = cuda_fail(e, "cudaEventElapsedTime");
+    if (s == BSA_OK) {
+      if (p->attn_path == 1) {
+        timings->summaries_ms = ms[0];
+        timings->select_ms = ms[1];
+        timings->pairing_ms = ms[2];
+        timings->attention_ms = ms[3];
+      } else {
+        timings->summaries_ms = ms[0];   // permute with the fused centroids
+        timings->select_ms = ms[1];
+        timings->attention_ms = ms[2];
+        timings->unpermute_ms = ms[3];
+      }
+      float total = 0.f;
+      if ((e = cudaEventElapsedTime(&total, t.ev[0], t.ev[t.n - 1])) != cudaSuccess)
+        s = cuda_fail(e, "cudaEventElapsedTime");
+      timings->total_ms = total;
+    }
+  }
+  destroy();
+  return s;
 }
 
 bsa_status bsa_kmax_for_union(bsa_plan_t p, bsa_select_mode mode, const double* param,

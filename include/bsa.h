@@ -493,6 +493,34 @@ bsa_status bsa_attention_paired(bsa_plan_t plan, const void* q, const void* k,
  * status word; returns BSA_OK or the recorded error. */
 bsa_status bsa_check_status(bsa_plan_t plan, void* stream);
 
+/* Device times of the phases of one bsa_forward call, in milliseconds (CUDA
+ * events recorded on the call's stream at each phase boundary).  SPADE Fig. 5
+ * splits one layer's sparse attention into "Pattern Search" and "Attention
+ * Computation"; here pattern search = summaries_ms + select_ms + pairing_ms. */
+typedef struct {
+  float summaries_ms;  /* tensor-core plans: the centroid pass over Q and K;
+                          other plans: the permute of Q, K, V with its centroids */
+  float select_ms;     /* scores, softmax and the Top-K / Top-P lists          */
+  float pairing_ms;    /* tile pairing (tensor-core plans; 0 when not run)     */
+  float attention_ms;  /* block-sparse attention (on tensor-core plans with the
+                          layout transform fused into its loads and stores)   */
+  float unpermute_ms;  /* inverse permute (other plans only)                   */
+  float total_ms;      /* first to last boundary                               */
+} bsa_timings_t;
+
+/* bsa_forward_timed — bsa_forward with per-phase device times.  Same
+ * arguments, outputs and errors as bsa_forward, plus `timings` (host
+ * pointer, must not be NULL; zeroed first).  Unlike bsa_forward it creates
+ * six CUDA events and synchronises on the last one before returning, so it
+ * is not for use inside a stream capture and costs a host round trip; the
+ * results are those of a plain bsa_forward call. */
+bsa_status bsa_forward_timed(bsa_plan_t plan, const void* q, const void* k,
+                             const void* v, bsa_select_mode mode,
+                             const double* param_per_head, int kmax, void* o,
+                             int32_t* idx_out, int32_t* cnt_out, void* ws,
+                             size_t ws_bytes, int32_t* dev_status, void* stream,
+                             bsa_timings_t* timings);
+
 /* bsa_plan_set_watchdog — bound of the tensor-core attention kernel's
  * in-kernel waits (failure detection; no counterpart on the pages, which
  * describe no failure handling).
