@@ -618,6 +618,13 @@ def run_ours(args, rank, world, local):
         return {n: sum(evs[si][ci].elapsed_time(evs[si][ci + 1]) for si in range(args.steps)) / args.steps
                 for ci, n in enumerate(names)}
 
+    # ---- the same split from inside the library: one bsa_forward_timed call
+    # (events at its phase boundaries), median of a few calls
+    splits = [plan.forward_timed(qd, kd, vd, w.mode, w.params, kmax=kmax, out=out, workspace=ws)[1]
+              for _ in range(5)]
+    library_split = {key: round(statistics.median(sp[key] for sp in splits), 4) for key in splits[0]}
+    plan.check_status()
+
     qc, kc = (torch.empty(plan.cent_shape, dtype=torch.float32, device=dev) for _ in range(2))
     S = lambda: bsa._stream(dev)
     if plan.info.attn_path == 1:
@@ -777,6 +784,7 @@ def run_ours(args, rank, world, local):
             "selected_pairs": pairs,
         },
         "phases_ms": {n: round(t, 4) for n, t in phase_ms.items()},
+        "phases_ms_in_forward": library_split,
         "phases_ms_unfused": {n: round(t, 4) for n, t in unfused.items()},
         "attn_tflops": round(attn_tf, 2),
         "attn_frac_of_peak": round(attn_tf / peak_tf, 4),
