@@ -299,6 +299,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // The two query tiles of this CTA (held in scalars: a runtime-indexed array
   // would live in local memory), and how many leading steps they share.
   int i0 = -1, i1 = -1, n0 = 0, n1 = 0, c_shared = 0;
+  int chunk = -1, kbase = 0;   // a text-chunk CTA of the paired schedule: its chunk and first key block
   long long bh0 = 0, bh1 = 0;
   const int32_t* list0;
   const int32_t* list1;
@@ -315,33 +316,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     list0 = a.idx + (bh0 * g.nb + (i0 >= 0 && i0 < g.nb ? i0 : 0)) * a.kmax;
     list1 = a.idx + (bh1 * g.nb + (i1 >= 0 && i1 < g.nb ? i1 : 0)) * a.kmax;
   } else {
-    // Paired schedule: CTA e covers the text pairs of every head first, then
-    // the video pairs; entry (h, t) names the two tiles and the shared count.
+    // Paired schedule, head-major: each head's group of CTAs opens with its
+    // text pairs split into text_chunks key chunks (one CTA each, about as
+    // long as a video pair), then its video pairs; entry (h, t) names the two
+    // tiles and the shared count.  A text chunk reads its head's K / V while
+    // the head's video pairs do, so one pass over K / V comes from DRAM.
     const int n_heads = map_count(a.map, g.B * g.Hd);
+    (void)n_heads;
     const int vpairs = a.pairs_per_head - a.text_pairs;
-    // Head-major order, each head's text pairs placed at the start of its own
-    // window so that they read its K / V while its video pairs do (one pass
-    // over the head's K / V from DRAM).  A text pair runs about text_lead
-    // head windows, so the text pairs of the last text_lead heads are issued
-    // together at the start of head n_heads - text_lead's window, early
-    // enough to finish with the rest of the launch.
-    const int tp = a.text_pairs, per = tp + vpairs;
-    const int lead = min(max(a.text_lead, 1), n_heads);
-    const int h_split = n_heads - lead;            // heads 0 .. h_split-1: own group
-    int e = blockIdx.x, m, t;
-    if (e < h_split * per) {
-      m = e / per;
-      t = e % per;
+    const int tp = a.text_pairs, nch = a.text_chunks, per = tp * nch + vpairs;
+    const int m = (int)blockIdx.x / per;
+    int t = (int)blockIdx.x % per;
+    if (t < tp * nch) {
+      chunk = t % nch;
+      t = t / nch;
     } else {
-      e -= h_split * per;
-      if (e < lead * tp) {
-        m = h_split + e / tp;
-        t = e % tp;
-      } else {
-        e -= lead * tp;
-        m = h_split + e / vpairs;
-        t = tp + e % vpairs;
-      }
+      t = tp + (t - tp * nch);
     }
     const long long bh = map_bh(a.map, m);
     const long long ent = bh * a.pairs_per_head + t;
@@ -349,16 +339,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bh0 = bh1 = bh;
     i0 = se.x;
     i1 = se.y;
-    if (i0 >= 0) n0 = list_length(g, a, bh, i0);
-    if (i1 >= 0) n1 = list_length(g, a, bh, i1);
-    c_shared = min(se.z, min(n0, n1));
+    if (chunk >= 0) {
+      // key blocks [chunk * len, ...) of the dense text rows, shared by both tiles
+      kbase = chunk * a.text_chunk_len;
+      const int len = min(a.text_chunk_len, nbk - kbase);
+      n0 = i0 >= 0 ? len : 0;
+      n1 = i1 >= 0 ? len : 0;
+      c_shared = min(n0, n1);   // a single-tile pair (odd text block count) shares nothing
+    } else {
+      if (i0 >= 0) n0 = list_length(g, a, bh, i0);
+      if (i1 >= 0) n1 = list_length(g, a, bh, i1);
+      c_shared = min(se.z, min(n0, n1));
+    }
     list0 = a.pair_lists + (ent * 2 + 0) * a.kmax;
     list1 = a.pair_lists + (ent * 2 + 1) * a.kmax;
   }
   // Key block of step s of tile x; -1 for an out-of-range list entry.
   auto block_at = [&](int x, int s) -> int {
     const int i = x ? i1 : i0;
-    const int j = i >= g.nb ? s : __ldg((x ? list1 : list0) + s);
+    const int j = i >= g.nb ? kbase + s : __ldg((x ? list1 : list0) + s);
     return (j >= 0 && j < nbk) ? j : -1;
   };
 
@@ -580,39 +579,66 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarO + x), 0, abort, lim));
         tc_fence_after();
       }
-      const uint4 qm = __ldg(reinterpret_cast<const uint4*>(a.masks) + qi);
-      const uint32_t qw4[4] = {qm.x, qm.y, qm.z, qm.w};
-      const bool slot_real = (qw4[r >> 5] >> (r & 31)) & 1u;
-      const bool row_valid = slot_real && ok && n > 0;
-      const float inv = (row_valid && l > 0.f) ? 1.f / l : 0.f;
-      // Blocked layout: every slot row is written (pad rows 0).  Original
-      // layout: each real slot's row goes to its token, pad slots are dropped.
-      long long orow_idx;
-      if (!ORIG) {
-        orow_idx = (qbh * nbk + qi) * 128 + r;
-      } else {
-        const long long tok = slot_token(g, qi, r);
-        orow_idx = tok >= 0 ? tok * g.Hd + (qbh % g.Hd) : -1;
-      }
-      uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + (orow_idx < 0 ? 0 : orow_idx) * HD);
+      if (chunk >= 0) {
+        // Text chunk: the unnormalised O row, the running max (log2 units)
+        // and the row sum go to the partial buffer; the merge pass combines
+        // the chunks of each text row.
+        const bool okr = ok && n > 0;
+        float* prow = a.part + ((((long long)qbh * g.nb_text + (qi - g.nb)) * a.text_chunks + chunk) * 128 + r) *
+                                   (long long)(HD + 4);
 #pragma unroll
-      for (int c0 = 0; c0 < HD; c0 += 32) {
-        uint32_t orr[32];
-        if (ok && n > 0) {
-          TMEM_LD32(tO + c0, orr);
-          TMEM_LD_WAIT(orr);
-        } else {
+        for (int c0 = 0; c0 < HD; c0 += 32) {
+          uint32_t orr[32];
+          if (okr) {
+            TMEM_LD32(tO + c0, orr);
+            TMEM_LD_WAIT(orr);
+          } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) orr[c] = 0u;
+            for (int c = 0; c < 32; ++c) orr[c] = 0u;
+          }
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4)
+            reinterpret_cast<uint4*>(prow + c0)[c4] =
+                make_uint4(orr[4 * c4], orr[4 * c4 + 1], orr[4 * c4 + 2], orr[4 * c4 + 3]);
         }
+        // an aborted CTA marks its rows (sum -1): the merge writes them as zeros
+        *reinterpret_cast<float4*>(prow + HD) =
+            make_float4(okr ? m_run : -INFINITY, okr ? l : -1.f, 0.f, 0.f);
+      } else {
+        const uint4 qm = __ldg(reinterpret_cast<const uint4*>(a.masks) + qi);
+        const uint32_t qw4[4] = {qm.x, qm.y, qm.z, qm.w};
+        const bool slot_real = (qw4[r >> 5] >> (r & 31)) & 1u;
+        const bool row_valid = slot_real && ok && n > 0;
+        const float inv = (row_valid && l > 0.f) ? 1.f / l : 0.f;
+        // Blocked layout: every slot row is written (pad rows 0).  Original
+        // layout: each real slot's row goes to its token, pad slots are dropped.
+        long long orow_idx;
+        if (!ORIG) {
+          orow_idx = (qbh * nbk + qi) * 128 + r;
+        } else {
+          const long long tok = slot_token(g, qi, r);
+          orow_idx = tok >= 0 ? tok * g.Hd + (qbh % g.Hd) : -1;
+        }
+        uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + (orow_idx < 0 ? 0 : orow_idx) * HD);
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(orr[8 * c8 + 0]) * inv, __uint_as_float(orr[8 * c8 + 1]) * inv);
-          v.y = pack_bf16x2(__uint_as_float(orr[8 * c8 + 2]) * inv, __uint_as_float(orr[8 * c8 + 3]) * inv);
-          v.z = pack_bf16x2(__uint_as_float(orr[8 * c8 + 4]) * inv, __uint_as_float(orr[8 * c8 + 5]) * inv);
-          v.w = pack_bf16x2(__uint_as_float(orr[8 * c8 + 6]) * inv, __uint_as_float(orr[8 * c8 + 7]) * inv);
-          if (orow_idx >= 0) orow[c0 / 8 + c8] = v;
+        for (int c0 = 0; c0 < HD; c0 += 32) {
+          uint32_t orr[32];
+          if (ok && n > 0) {
+            TMEM_LD32(tO + c0, orr);
+            TMEM_LD_WAIT(orr);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) orr[c] = 0u;
+          }
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(orr[8 * c8 + 0]) * inv, __uint_as_float(orr[8 * c8 + 1]) * inv);
+            v.y = pack_bf16x2(__uint_as_float(orr[8 * c8 + 2]) * inv, __uint_as_float(orr[8 * c8 + 3]) * inv);
+            v.z = pack_bf16x2(__uint_as_float(orr[8 * c8 + 4]) * inv, __uint_as_float(orr[8 * c8 + 5]) * inv);
+            v.w = pack_bf16x2(__uint_as_float(orr[8 * c8 + 6]) * inv, __uint_as_float(orr[8 * c8 + 7]) * inv);
+            if (orow_idx >= 0) orow[c0 / 8 + c8] = v;
+          }
         }
       }
     }
@@ -662,11 +688,63 @@ cudaError_t launch_attn_tc_orig(const Geo& g, const AttnArgs& a, const TileMaps&
                                 cudaStream_t st) {
   const int tiles = map_count(a.map, g.Hd) * (g.nb + g.nb_text);
   if (tiles == 0 || g.B != 1) return g.B != 1 ? cudaErrorInvalidValue : cudaSuccess;
-  // paired schedule: one CTA per entry (a head with an odd tile count has a
-  // single-tile entry)
-  const int ctas = a.pair_sched ? map_count(a.map, g.Hd) * a.pairs_per_head : (tiles + 1) / 2;
+  // paired schedule: one CTA per video pair (a head with an odd tile count
+  // has a single-tile entry) and per key chunk of each text pair
+  const int ctas = a.pair_sched ? map_count(a.map, g.Hd) *
+                                      (a.pairs_per_head - a.text_pairs + a.text_pairs * a.text_chunks)
+                                : (tiles + 1) / 2;
   return g.D == 128 ? launch_tc_t<128, true>(g, a, maps, ctas, st)
                     : launch_tc_t<64, true>(g, a, maps, ctas, st);
+}
+
+// Merge of the key-chunk partials of the text rows (SPADE §3.3 (3)'s online
+// softmax, finished across chunks): for a row with partials (O_c, m_c, l_c),
+// M = max_c m_c, w_c = 2^(m_c - M), output = sum_c w_c O_c / sum_c w_c l_c,
+// rounded to bf16 (the same quotient the one-CTA path forms, with the sums
+// regrouped).  One warp per text row, lanes over the head dimension.
+constexpr int kMergeWarps = 8;
+
+template <int HD>
+__global__ void __launch_bounds__(kMergeWarps * 32) text_merge_kernel(Geo g, MergeArgs a) {
+  constexpr int kPer = HD / 32;                       // columns per lane
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long u = (long long)blockIdx.x * kMergeWarps + warp;   // text token
+  if (u >= g.n_text) return;
+  const long long bh = map_bh(a.map, blockIdx.y);
+  const int tb = (int)(u / 128), r = (int)(u % 128);
+  const long long stride_c = 128ll * (HD + 4);
+  const float* base = a.part + (((bh * g.nb_text + tb) * a.text_chunks) * 128 + r) * (long long)(HD + 4);
+  float M = -INFINITY;
+  for (int c = 0; c < a.text_chunks; ++c) M = fmaxf(M, base[c * stride_c + HD]);
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  float lsum = 0.f;
+  bool aborted = false;
+  for (int c = 0; c < a.text_chunks; ++c) {
+    const float* pc = base + c * stride_c;
+    const float mc = pc[HD];
+    aborted = aborted || pc[HD + 1] < 0.f;
+    const float w = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+    lsum = fmaf(w, pc[HD + 1], lsum);
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] = fmaf(w, pc[kPer * lane + e], acc[e]);
+  }
+  const float inv = (lsum > 0.f && !aborted) ? 1.f / lsum : 0.f;
+  __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) +
+                        ((g.n_video + u) * g.Hd + (bh % g.Hd)) * HD + kPer * lane;
+#pragma unroll
+  for (int e = 0; e < kPer; e += 2)
+    *reinterpret_cast<uint32_t*>(orow + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+}
+
+cudaError_t launch_text_merge(const Geo& g, const MergeArgs& a, cudaStream_t st) {
+  const int heads = map_count(a.map, g.Hd);
+  if (g.n_text == 0 || heads == 0 || g.B != 1) return g.B != 1 ? cudaErrorInvalidValue : cudaSuccess;
+  const dim3 grid((unsigned)((g.n_text + kMergeWarps - 1) / kMergeWarps), (unsigned)heads);
+  if (g.D == 128) text_merge_kernel<128><<<grid, kMergeWarps * 32, 0, st>>>(g, a);
+  else text_merge_kernel<64><<<grid, kMergeWarps * 32, 0, st>>>(g, a);
+  return cudaGetLastError();
 }
 
 }  // namespace bsa

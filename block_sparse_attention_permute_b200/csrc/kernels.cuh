@@ -95,10 +95,24 @@ struct AttnArgs {
   const int32_t* pair_sched;
   const int32_t* pair_lists;
   int pairs_per_head, text_pairs;
-  int text_lead;          // head windows a text pair spans (its position in the order)
+  // Text pairs of the paired schedule split into text_chunks key chunks of
+  // text_chunk_len blocks; a chunk's partial rows go to
+  //   part[((((bh * nb_text + (i - nb)) * text_chunks + c) * 128 + r) * (D + 4) + d]
+  //   d < D: unnormalised O, d = D: running max (log2 units), d = D + 1: row sum
+  float* part;
+  int text_chunks, text_chunk_len;
   // divisors of the per-copy block coordinates (nbx, nby, Hd), so that the
   // copy-issuing thread divides without the MUFU unit
   FastDiv div_nbx, div_nby, div_hd;
+};
+
+// Merge of the text rows' key-chunk partials into the output (original
+// layout, one batch element per launch).
+struct MergeArgs {
+  const float* part;      // as AttnArgs::part
+  void* o;                // [Ntot, Hd, D] of the batch element
+  int text_chunks;
+  HeadMap map;            // heads of the launch (n = 0: all)
 };
 
 // Pairing of the query tiles of each (b, h) into CTA pairs that share key
@@ -143,6 +157,7 @@ cudaError_t launch_attn_simt(const Geo& g, bool is_bf16, const AttnArgs& a, cuda
 cudaError_t launch_attn_tc(const Geo& g, const AttnArgs& a, const TileMaps& maps, cudaStream_t st);
 cudaError_t launch_attn_tc_orig(const Geo& g, const AttnArgs& a, const TileMaps& maps,
                                 cudaStream_t st);
+cudaError_t launch_text_merge(const Geo& g, const MergeArgs& a, cudaStream_t st);
 cudaError_t launch_pool_orig(const Geo& g, bool is_bf16, const GatherArgs& a, cudaStream_t st);
 
 }  // namespace bsa

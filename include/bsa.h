@@ -466,7 +466,12 @@ bsa_status bsa_forward_grouped(const bsa_plan_t* plans, int n_plans,
  * fetches each shared K and V tile once for both tiles.  bsa_forward does
  * both on tensor-core plans.  Lists must be as bsa_select writes them
  * (ascending video blocks, then every text block).  The result equals
- * bsa_attention_orig up to the rounding of the reordered sums. */
+ * bsa_attention_orig up to the rounding of the reordered sums.  The text
+ * query tiles (dense rows) run as key chunks about one list long, each in
+ * its head's group of CTAs; their partial rows (unnormalised output, running
+ * maximum, row sum) are kept in the tail of the pairing workspace and merged
+ * by a second launch (SPADE §3.3 (3)'s online softmax finished across
+ * chunks). */
 
 /* bsa_pair_workspace_size — bytes of the pairing workspace (0 off the
  * tensor-core path). */
@@ -482,10 +487,11 @@ bsa_status bsa_pair_tiles(bsa_plan_t plan, const int32_t* idx,
 
 /* bsa_attention_paired — bsa_attention_orig on the schedule bsa_pair_tiles
  * wrote into ws from the same idx / cnt (same plan limits as
- * bsa_pair_tiles). */
+ * bsa_pair_tiles).  It writes the text rows' partials into the workspace's
+ * tail (the schedule itself is only read). */
 bsa_status bsa_attention_paired(bsa_plan_t plan, const void* q, const void* k,
                                 const void* v, const int32_t* idx,
-                                const int32_t* cnt, int kmax, const void* ws,
+                                const int32_t* cnt, int kmax, void* ws,
                                 size_t ws_bytes, void* o, int32_t* dev_status,
                                 void* stream);
 
