@@ -442,7 +442,7 @@ def time_workload(bsa, name, dev, barrier, args, cache, peak_burst, peak_sust):
     e1.record(stream)
     barrier()
     est_ms = e0.elapsed_time(e1) / 3
-    n = int(min(400, max(args.steps, -(-600.0 // max(est_ms, 1e-3)))))
+    n = int(min(20000, max(args.steps, -(-600.0 // max(est_ms, 1e-3)))))
     pairs = effective_pairs(plan, idx, cnt)
     flops = 4.0 * pairs * w.D
     with ClockSampler(dev.index) as clk:
