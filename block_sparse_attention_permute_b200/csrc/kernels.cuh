@@ -142,7 +142,7 @@ cudaError_t launch_unpermute(const Geo& g, bool is_bf16, const GatherArgs& a, cu
 cudaError_t launch_pool(const Geo& g, bool is_bf16, const GatherArgs& a, cudaStream_t st);
 cudaError_t launch_sics_schemes(const SchemeArgs& a, bool is_bf16, cudaStream_t st);
 // select.cu
-size_t select_smem_bytes(int nb, int D, int rows = 16);   // rows: query blocks per CTA
+size_t select_smem_bytes(int nb, int D, int rows = 16, int kpt = 2);   // rows: query blocks per CTA; kpt: keys per thread
 cudaError_t launch_select(const Geo& g, const SelectArgs& a, cudaStream_t st);
 cudaError_t launch_intra_select(const Geo& g, const IntraArgs& a, cudaStream_t st);
 // pair.cu

@@ -23,15 +23,14 @@ namespace bsa {
 
 
 constexpr int kSelRows = 16;      // query-block rows per CTA (8 for long rows, see launch_select_t)
-constexpr int kSelKeys = 256;     // key blocks per score chunk
 constexpr int kSelDChunk = 8;    // head-dim slice of a key chunk held in shared memory
 constexpr int kSelBufs = 2;      // key-chunk buffers (2: the next chunk lands while one is used)
 constexpr int kSelKS = kSelDChunk + 4;   // padded chunk row: conflict-free float4 reads
 constexpr int kSelThreads = 256;  // 8 warps
 
 // query summaries, the key-chunk buffers, the score rows
-size_t select_smem_bytes(int nb, int D, int rows) {
-  return sizeof(float) * ((size_t)rows * D + kSelBufs * (size_t)kSelKeys * kSelKS + (size_t)rows * nb);
+size_t select_smem_bytes(int nb, int D, int rows, int kpt) {
+  return sizeof(float) * ((size_t)rows * D + kSelBufs * (size_t)(128 * kpt) * kSelKS + (size_t)rows * nb);
 }
 
 __device__ __forceinline__ uint32_t order_key(float s) {
@@ -254,14 +253,18 @@ __device__ __forceinline__ float box_max_product(float aM, float am, float bM, f
 
 // D = length of the stored summary vectors (head_dim for MEAN, 2 * head_dim
 // for the (max, min) boxes of DSA and DSA2).
-template <int D, int EST, int ROWS, int KMAX>
+// KPT: keys per thread in a score chunk of 128 * KPT key blocks (2: chunks
+// of 256; 3 where a row of nb keys pads less in chunks of 384, e.g. Wan's
+// nb = 336: 48 idle key slots instead of 176, 15-17 % less selection time).
+template <int D, int EST, int ROWS, int KMAX, int KPT>
 __global__ void __launch_bounds__(kSelThreads, KMAX == 16 ? 3 : 2)
     select_kernel(Geo g, SelectArgs a) {
   constexpr int RPT = ROWS / 2;                     // rows per thread in phase 1
+  constexpr int KC = 128 * KPT;                     // key blocks per score chunk
   extern __shared__ __align__(16) float sm[];
   float* qs = sm;                                   // [ROWS][D]
-  float* ks = qs + ROWS * D;                        // [kSelBufs][kSelKeys][kSelKS]
-  float* sc = ks + kSelBufs * kSelKeys * kSelKS;    // [ROWS][nb]
+  float* ks = qs + ROWS * D;                        // [kSelBufs][KC][kSelKS]
+  float* sc = ks + kSelBufs * KC * kSelKS;          // [ROWS][nb]
   const int nb = g.nb;
   const int bhi = map_bh(a.map, (int)blockIdx.z * g.Hd + (int)blockIdx.y);
   const int h = bhi % g.Hd, b = bhi / g.Hd;
@@ -270,8 +273,8 @@ __global__ void __launch_bounds__(kSelThreads, KMAX == 16 ? 3 : 2)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   // ---- phase 1: scores of ROWS query blocks against all key blocks ----
-  // Thread (ty, tx) accumulates rows RPT ty .. RPT ty + RPT - 1 against keys tx and tx+128 of
-  // each 256-key chunk; the chunk's keys pass through shared memory 8
+  // Thread (ty, tx) accumulates rows RPT ty .. RPT ty + RPT - 1 against keys tx + 128 k
+  // (k < KPT) of each KC-key chunk; the chunk's keys pass through shared memory 8
   // dimensions at a time (double-buffered).  Each dot product is one fma chain over d in
   // ascending order, the same as a plain sequential loop.
   if (EST == kEstDsa) {
@@ -296,16 +299,16 @@ __global__ void __launch_bounds__(kSelThreads, KMAX == 16 ? 3 : 2)
     }
   }
   const int ty = tid / 128, tx = tid % 128;
-  // The key chunks (kSelKeys key blocks x kSelDChunk dimensions) are visited
+  // The key chunks (KC key blocks x kSelDChunk dimensions) are visited
   // j0-major; chunk c + 1 is copied with cp.async into the other buffer while
   // chunk c is used.  Rows past nb are zero-filled.
   constexpr int kDChunks = D / kSelDChunk;
-  const int n_chunks = ((nb + kSelKeys - 1) / kSelKeys) * kDChunks;
+  const int n_chunks = ((nb + KC - 1) / KC) * kDChunks;
   const float* kc_bh = a.kc + bh * nb * D;
   auto issue_chunk = [&](int c) {
-    const int j0 = (c / kDChunks) * kSelKeys, d0 = (c % kDChunks) * kSelDChunk;
-    float* buf = ks + (c % kSelBufs) * kSelKeys * kSelKS;
-    for (int e = tid; e < kSelKeys * (kSelDChunk / 4); e += kSelThreads) {
+    const int j0 = (c / kDChunks) * KC, d0 = (c % kDChunks) * kSelDChunk;
+    float* buf = ks + (c % kSelBufs) * KC * kSelKS;
+    for (int e = tid; e < KC * (kSelDChunk / 4); e += kSelThreads) {
       const int jj = e / (kSelDChunk / 4), d4 = e % (kSelDChunk / 4);
       const bool ok = j0 + jj < nb;
       cp_async16(smem_addr(buf + jj * kSelKS + 4 * d4),
@@ -314,12 +317,14 @@ __global__ void __launch_bounds__(kSelThreads, KMAX == 16 ? 3 : 2)
     cp_async_commit();
   };
   if (kSelBufs == 2) issue_chunk(0);
-  float acc[RPT][2];
+  float acc[RPT][KPT];
   for (int c = 0; c < n_chunks; ++c) {
-    const int j0 = (c / kDChunks) * kSelKeys, d0 = (c % kDChunks) * kSelDChunk;
+    const int j0 = (c / kDChunks) * KC, d0 = (c % kDChunks) * kSelDChunk;
     if (d0 == 0) {
 #pragma unroll
-      for (int r = 0; r < RPT; ++r) acc[r][0] = acc[r][1] = 0.f;
+      for (int r = 0; r < RPT; ++r)
+#pragma unroll
+        for (int kp = 0; kp < KPT; ++kp) acc[r][kp] = 0.f;
     }
     if (kSelBufs == 1) {
       issue_chunk(c);
@@ -331,37 +336,37 @@ __global__ void __launch_bounds__(kSelThreads, KMAX == 16 ? 3 : 2)
       cp_async_wait<0>();
     }
     __syncthreads();   // chunk c (and, at c = 0, the query summaries) visible
-    const float* kb = ks + (c % kSelBufs) * kSelKeys * kSelKS;
+    const float* kb = ks + (c % kSelBufs) * KC * kSelKS;
 #pragma unroll
     for (int d4 = 0; d4 < kSelDChunk / 4; ++d4) {
-      const float4 k0 = *reinterpret_cast<const float4*>(kb + tx * kSelKS + 4 * d4);
-      const float4 k1 = *reinterpret_cast<const float4*>(kb + (tx + 128) * kSelKS + 4 * d4);
+      float4 kv[KPT];
+#pragma unroll
+      for (int kp = 0; kp < KPT; ++kp)
+        kv[kp] = *reinterpret_cast<const float4*>(kb + (tx + 128 * kp) * kSelKS + 4 * d4);
 #pragma unroll
       for (int r = 0; r < RPT; ++r) {
         const float4 qv = *reinterpret_cast<const float4*>(qs + (RPT * ty + r) * D + d0 + 4 * d4);
-        if (EST == kEstDsa2) {
-          acc[r][0] += box_max_product(qv.x, qv.y, k0.x, k0.y);
-          acc[r][0] += box_max_product(qv.z, qv.w, k0.z, k0.w);
-          acc[r][1] += box_max_product(qv.x, qv.y, k1.x, k1.y);
-          acc[r][1] += box_max_product(qv.z, qv.w, k1.z, k1.w);
-          continue;
+#pragma unroll
+        for (int kp = 0; kp < KPT; ++kp) {
+          if (EST == kEstDsa2) {
+            acc[r][kp] += box_max_product(qv.x, qv.y, kv[kp].x, kv[kp].y);
+            acc[r][kp] += box_max_product(qv.z, qv.w, kv[kp].z, kv[kp].w);
+            continue;
+          }
+          acc[r][kp] = fmaf(qv.x, kv[kp].x, acc[r][kp]);
+          acc[r][kp] = fmaf(qv.y, kv[kp].y, acc[r][kp]);
+          acc[r][kp] = fmaf(qv.z, kv[kp].z, acc[r][kp]);
+          acc[r][kp] = fmaf(qv.w, kv[kp].w, acc[r][kp]);
         }
-        acc[r][0] = fmaf(qv.x, k0.x, acc[r][0]);
-        acc[r][0] = fmaf(qv.y, k0.y, acc[r][0]);
-        acc[r][0] = fmaf(qv.z, k0.z, acc[r][0]);
-        acc[r][0] = fmaf(qv.w, k0.w, acc[r][0]);
-        acc[r][1] = fmaf(qv.x, k1.x, acc[r][1]);
-        acc[r][1] = fmaf(qv.y, k1.y, acc[r][1]);
-        acc[r][1] = fmaf(qv.z, k1.z, acc[r][1]);
-        acc[r][1] = fmaf(qv.w, k1.w, acc[r][1]);
       }
     }
     if (d0 + kSelDChunk == D) {
 #pragma unroll
-      for (int r = 0; r < RPT; ++r) {
-        if (j0 + tx < nb) sc[(RPT * ty + r) * nb + j0 + tx] = acc[r][0] * a.scale + 0.0f;
-        if (j0 + tx + 128 < nb) sc[(RPT * ty + r) * nb + j0 + tx + 128] = acc[r][1] * a.scale + 0.0f;
-      }
+      for (int r = 0; r < RPT; ++r)
+#pragma unroll
+        for (int kp = 0; kp < KPT; ++kp)
+          if (j0 + tx + 128 * kp < nb)
+            sc[(RPT * ty + r) * nb + j0 + tx + 128 * kp] = acc[r][kp] * a.scale + 0.0f;
     }
     __syncthreads();   // buffer (c & 1) is refilled by the copy issued next iteration
   }
@@ -465,16 +470,16 @@ cudaError_t launch_intra_select(const Geo& g, const IntraArgs& a, cudaStream_t s
   return cudaGetLastError();
 }
 
-template <int D, int EST, int ROWS, int KMAX>
+template <int D, int EST, int ROWS, int KMAX, int KPT = 2>
 static cudaError_t launch_select_rows(const Geo& g, const SelectArgs& a, cudaStream_t st) {
-  const size_t smem = select_smem_bytes(g.nb, D, ROWS);
+  const size_t smem = select_smem_bytes(g.nb, D, ROWS, KPT);
   // with a head map, y enumerates its pairs (z = 1) and the kernel reads
   // map_bh(y); without one, y = h and z = b
   dim3 grid((g.nb + ROWS - 1) / ROWS, a.map.n ? a.map.n : g.Hd, a.map.n ? 1 : g.B);
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<D, EST, ROWS, KMAX>,
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<D, EST, ROWS, KMAX, KPT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  select_kernel<D, EST, ROWS, KMAX><<<grid, kSelThreads, smem, st>>>(g, a);
+  select_kernel<D, EST, ROWS, KMAX, KPT><<<grid, kSelThreads, smem, st>>>(g, a);
   return cudaGetLastError();
 }
 
@@ -486,6 +491,9 @@ template <int D, int EST>
 static cudaError_t launch_select_t(const Geo& g, const SelectArgs& a, cudaStream_t st) {
   constexpr size_t kTwoPerSm = 112 * 1024;
   const bool rows16 = select_smem_bytes(g.nb, D, kSelRows) <= kTwoPerSm;
+  // rows in (256, 384] (Wan's 336 blocks) waste less in one chunk of 384 keys
+  const bool kpt3 = g.nb > 256 && g.nb <= 384 && select_smem_bytes(g.nb, D, kSelRows, 3) <= kTwoPerSm;
+  if (g.nb <= 32 * 16 && kpt3) return launch_select_rows<D, EST, kSelRows, 16, 3>(g, a, st);
   if (g.nb <= 32 * 16 && rows16) return launch_select_rows<D, EST, kSelRows, 16>(g, a, st);
   if (g.nb <= 32 * 32 && rows16) return launch_select_rows<D, EST, kSelRows, 32>(g, a, st);
   if (g.nb <= 32 * kKeysPerLane)
