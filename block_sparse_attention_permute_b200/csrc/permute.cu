@@ -13,6 +13,8 @@
 // covers two 256-byte rows per instruction).  The slot -> token map of the
 // block is decoded once into shared memory.  HBM-bound: each byte is read
 // once and written once.
+#include <cmath>
+
 #include "kernels.cuh"
 
 namespace bsa {
@@ -224,20 +226,22 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(Geo g, GatherArg
 // blocked-layout pool.
 constexpr int kColThreads = 128;
 
-template <int D>
-__global__ void __launch_bounds__(kColThreads) pool_cols_kernel(Geo g, GatherArgs a) {
+// THREADS / V heads per CTA (the launcher picks the count that fills the
+// GPU's CTA slots best); a thread's sum is the same for every count.
+template <int D, int THREADS>
+__global__ void __launch_bounds__(THREADS) pool_cols_kernel(Geo g, GatherArgs a) {
   using T = __nv_bfloat16;
   constexpr int E = 8;                      // bf16 elements per 16-byte vector
   constexpr int V = D / E;                  // vectors per row
   constexpr int R = kGatherThreads / V;     // row groups, as in gather_block
   constexpr int M = 128 / R;                // rows per group
-  constexpr int HG = kColThreads / V;       // heads per CTA
+  constexpr int HG = THREADS / V;           // heads per CTA
   __shared__ int s_tok[128];
   const int j = blockIdx.x, t = blockIdx.z;
   const int p = blockIdx.y * HG + (int)threadIdx.x / V, vec = (int)threadIdx.x % V;
   const void* src_ptr = t == 0 ? a.src[0] : t == 1 ? a.src[1] : a.src[2];
   float* cent = t == 0 ? a.cent[0] : t == 1 ? a.cent[1] : a.cent[2];
-  s_tok[threadIdx.x] = (int)slot_token(g, j, threadIdx.x);
+  for (int x = threadIdx.x; x < 128; x += THREADS) s_tok[x] = (int)slot_token(g, j, x);
   __syncthreads();
   if (p >= map_count(a.map, g.B * g.Hd) || cent == nullptr) return;
   const int bh = map_bh(a.map, p), b = bh / g.Hd, h = bh % g.Hd;
@@ -550,6 +554,19 @@ cudaError_t launch_unpermute(const Geo& g, bool is_bf16, const GatherArgs& a, cu
                  : launch_gather_t<float, kUnpermute>(g, a, nblocks, st);
 }
 
+// Multiprocessors of the current device (queried once per device).
+static int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    cached[dev] = (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+                      ? n : 148;
+  }
+  return cached[dev];
+}
+
 // Centroids of the video blocks straight from the original layout (the
 // summarizer pass of the fused forward, which never materialises the blocked
 // tensors).
@@ -564,9 +581,34 @@ cudaError_t launch_pool_orig(const Geo& g, bool is_bf16, const GatherArgs& a, cu
     if (extras) {
       if (g.D == 128) pool_cols_extras_kernel<128><<<grid, kColThreads, 0, st>>>(g, a);
       else pool_cols_extras_kernel<64><<<grid, kColThreads, 0, st>>>(g, a);
+      return cudaGetLastError();
+    }
+    // Heads per CTA: 128 threads (8 CTAs per SM at 64 registers a thread,
+    // the most loads in flight) unless 192 or 256 threads (5 or 4 CTAs per
+    // SM) need fewer waves of CTA slots.  Wan2.1-1.3B's 12 heads: 192
+    // threads, one head group, 672 CTAs in one wave of 740 slots instead of
+    // 1344 in 1184 (centroids 43 -> 37 us); HunyuanVideo, Wan2.1-14B and
+    // Long keep 128 (as many waves either way; 192 measured slower there).
+    const int V = g.D / 8;
+    const int sms = sm_count();
+    auto waves = [&](int threads) {
+      const int hgc = threads / V;
+      const long long ctas = (long long)g.nb * ((pairs + hgc - 1) / hgc) * a.ntensors;
+      const long long slots = (long long)sms * (65536 / (threads * 64));
+      return (ctas + slots - 1) / slots;
+    };
+    int best = 128;
+    for (int threads : {192, 256})
+      if (waves(threads) < waves(best)) best = threads;
+    const dim3 grid_b(g.nb, (pairs + best / V - 1) / (best / V), a.ntensors);
+    if (g.D == 128) {
+      if (best == 192) pool_cols_kernel<128, 192><<<grid_b, 192, 0, st>>>(g, a);
+      else if (best == 256) pool_cols_kernel<128, 256><<<grid_b, 256, 0, st>>>(g, a);
+      else pool_cols_kernel<128, 128><<<grid_b, 128, 0, st>>>(g, a);
     } else {
-      if (g.D == 128) pool_cols_kernel<128><<<grid, kColThreads, 0, st>>>(g, a);
-      else pool_cols_kernel<64><<<grid, kColThreads, 0, st>>>(g, a);
+      if (best == 192) pool_cols_kernel<64, 192><<<grid_b, 192, 0, st>>>(g, a);
+      else if (best == 256) pool_cols_kernel<64, 256><<<grid_b, 256, 0, st>>>(g, a);
+      else pool_cols_kernel<64, 128><<<grid_b, 128, 0, st>>>(g, a);
     }
     return cudaGetLastError();
   }
