@@ -350,6 +350,52 @@ def test_aggregation_score_and_scheme_choice():
     assert np.all(scores[choice[0], 0, np.arange(3)] >= scores.max(0)[0] - 1e-12)
 
 
+def test_aggregation_score_closed_forms():
+    """AS on inputs built so that every block's sum of unit vectors is known:
+    the tokens point along coordinate axes (each scaled by a random positive
+    factor, which normalisation removes), so a block's SICS is |sum of unit
+    vectors|^2 = sum over axes of (signed token count along that axis)^2
+    (SPADE §3.2, Eq. (4), diagonal included), and AS (Eq. (3)) sums it over the
+    blocks.  Each head's axis pattern follows one blocking scheme, so the
+    scheme choice is known too."""
+    T, H, W, D = 4, 8, 8, 16
+    base = dict(B=1, T=T, H=H, W=W, Hd=5, D=D, n_text=0)
+    geoms = [orc.Geometry(bf=1, br=8, bc=8, **base),     # one frame per block
+             orc.Geometry(bf=4, br=4, bc=4, **base),     # 4x4x4 cubes
+             orc.Geometry(bf=2, br=2, bc=16, **base)]    # 2x2x16, ragged in W (8 real columns)
+    rng = np.random.default_rng(5)
+    x = np.zeros((1, T * H * W, 5, D), dtype=np.float32)
+    for t in range(T):
+        for y in range(H):
+            for c in range(W):
+                n = (t * H + y) * W + c
+                s = rng.uniform(0.25, 4.0, size=5).astype(np.float32)
+                x[0, n, 0, t] = s[0]                                   # axis = frame
+                x[0, n, 1, 2 * (y // 4) + c // 4] = s[1]               # axis = (y, x) quadrant
+                x[0, n, 2, 4 * (t // 2) + y // 2] = s[2]               # axis = (frame pair, row pair)
+                x[0, n, 3, t] = s[3] * (1 if c % 2 == 0 else -1)       # frame axis, sign by column parity
+                if t > 0:
+                    x[0, n, 4, t] = s[4]                               # head 0's pattern, frame 0 zero
+    # per scheme (rows) and head (columns), from the counts above:
+    #  head 0: frame blocks hold 64 tokens on one axis (4 * 64^2); a cube holds
+    #          16 per frame on 4 axes (4 blocks * 4 * 16^2); a 2x2x8 block 16 on
+    #          each of 2 axes (8 blocks * 2 * 16^2)
+    #  head 1: a frame holds 16 tokens on each of 4 axes; a cube 64 on one axis;
+    #          a 2x2x8 block 16 on each of 2 axes
+    #  head 2: a frame holds 16 on each of 4 axes; a cube 16 on each of 4 axes;
+    #          a 2x2x8 block 32 on one axis
+    #  head 3: every block holds as many -e as +e tokens on each axis: 0
+    #  head 4: head 0 without frame 0 (zero vectors count for nothing):
+    #          3 * 64^2; 4 cubes * 3 * 16^2; 4 blocks * 16^2 + 4 blocks * 2 * 16^2
+    expect = np.array([[16384, 4096, 4096, 0, 12288],
+                       [4096, 16384, 4096, 0, 3072],
+                       [4096, 4096, 8192, 0, 3072]], dtype=np.float64)
+    choice, scores = orc.choose_scheme(geoms, x)
+    np.testing.assert_allclose(scores[:, 0, :], expect, rtol=1e-12, atol=1e-9)
+    # head 3 is a three-way tie: the lowest scheme index
+    assert list(choice[0]) == [0, 1, 2, 0, 0]
+
+
 # ------------------------------------------------ mask-union pins (SPADE §3.3)
 def _inter_sets(g, p, mode, params):
     idx, cnt, _ = orc.select(g, p, mode, params)
