@@ -474,7 +474,8 @@ def time_workload(bsa, name, dev, barrier, args, cache, peak_burst, peak_sust):
         else:
             calls += [lambda: L.bsa_attention_orig(plan._h, P(qd), P(kd), P(vd), P(idx), P(cnt), kmax,
                                                    P(out), None, S())]
-        launches = 3 + (4 if paired else 0) + (1 if paired and plan.info.nb_text > 0 else 0)
+        # per bsa_forward step: centroids, select, 2 pairing kernels, attention, text merge
+        launches = 3 + (2 if paired else 0) + (1 if paired and plan.info.nb_text > 0 else 0)
     else:
         qb, kb, vb, ob = (torch.empty(plan.blk_shape, dtype=plan.dtype, device=dev) for _ in range(4))
         names = ["permute", "select", "attention", "unpermute"]
@@ -502,7 +503,14 @@ def time_workload(bsa, name, dev, barrier, args, cache, peak_burst, peak_sust):
     ph = {nm: sum(evs[si][ci].elapsed_time(evs[si][ci + 1]) for si in range(m)) / m
           for ci, nm in enumerate(names)}
     attn_tf = flops / (ph["attention"] * 1e-3) / 1e12
-    pre = ph.get("centroids", ph.get("permute", 0.0)) + ph["select"] + ph.get("pairing", 0.0)
+    pre_calls = ph.get("centroids", ph.get("permute", 0.0)) + ph["select"] + ph.get("pairing", 0.0)
+    # the same split inside bsa_forward as it runs (events at its phase
+    # boundaries; the selection there also hands the pairing its bit sets)
+    splits = [plan.forward_timed(qd, kd, vd, w.mode, w.params, kmax=kmax, out=out, workspace=ws)[1]
+              for _ in range(max(5, min(m, 15)))]
+    plan.check_status()
+    fs = {key: statistics.median(sp[key] for sp in splits) for key in splits[0]}
+    pre = fs["summaries_ms"] + fs["select_ms"] + fs["pairing_ms"]
     res = {
         "shape": workload_config(w)["shape"],
         "selection": workload_config(w)["selection"],
@@ -514,7 +522,10 @@ def time_workload(bsa, name, dev, barrier, args, cache, peak_burst, peak_sust):
         "phases_ms": {nm: round(t, 4) for nm, t in ph.items()},
         "attn_ms": round(ph["attention"], 4),
         "attn_tflops": round(attn_tf, 2),
-        "pre_attention_share": round(pre / ph["attention"], 4),
+        "phases_ms_in_forward": {key: round(t, 4) for key, t in fs.items()},
+        "pre_attention_share": round(pre / fs["attention_ms"], 4),
+        "pre_attention_share_of": "summaries + select + pairing over attention, inside bsa_forward_timed",
+        "pre_attention_share_calls": round(pre_calls / ph["attention"], 4),
         "pre_attention_phases": [nm for nm in names if nm not in ("attention", "unpermute")],
         "clocks": clocks,
         "gpu_launches_per_step": launches,
@@ -792,6 +803,9 @@ def run_ours(args, rank, world, local):
         "permute_select_share_of_attn": round(
             (phase_ms.get("centroids", phase_ms.get("permute", 0.0)) + phase_ms["select"]
              + phase_ms.get("pairing", 0.0)) / phase_ms["attention"], 4),
+        "permute_select_share_of_attn_in_forward": round(
+            (library_split["summaries_ms"] + library_split["select_ms"] + library_split["pairing_ms"])
+            / library_split["attention_ms"], 4),
         "permute_select_share_of_attn_unfused": round(
             (unfused["permute"] + unfused["select"]) / unfused["attention"], 4),
         "roofline": {
@@ -821,11 +835,12 @@ def run_ours(args, rank, world, local):
         "scheme_generation": dict(scheme, share_of_attn=round(scheme["ms"] / phase_ms["attention"], 4),
                                   frac=round(scheme["achieved_gbs"] / hbm_gbs, 4),
                                   peak_gbs=hbm_gbs, bound="hbm"),
-        # per bsa_forward step, tensor-core plans: centroids, select, 4 pairing
-        # kernels (bit sets, candidates, matching, lists; none beyond 1536 video
-        # blocks), attention, and with text tokens the merge of the text
-        # chunks; other plans: permute, select, attention, unpermute
-        "gpu_launches": ((3 + (4 if plan.info.nb <= 1536 else 0)
+        # per bsa_forward step, tensor-core plans: centroids, select (which also
+        # writes the lists' bit sets), 2 pairing kernels (candidates; matching
+        # with the reordered lists; none beyond 1536 video blocks), attention,
+        # and with text tokens the merge of the text chunks; other plans:
+        # permute, select, attention, unpermute
+        "gpu_launches": ((3 + (2 if plan.info.nb <= 1536 else 0)
                           + (1 if plan.info.nb <= 1536 and plan.info.nb_text > 0 else 0))
                          if plan.info.attn_path == 1 else 4) * args.steps,
         "clocks": clocks,

@@ -234,7 +234,7 @@ bsa_status run_select(const bsa_plan_s* p, const float* qc, const float* kc, bsa
                       const double* param, int kmax, int32_t* idx, int32_t* cnt, float* scores,
                       cudaStream_t st, const UnionOpts* uo = nullptr, const float* intra_scores = nullptr,
                       uint32_t* bits = nullptr, int est = bsa::kEstMean,
-                      const bsa::HeadMap* map = nullptr) {
+                      const bsa::HeadMap* map = nullptr, uint32_t* list_bits = nullptr) {
   int need = 0;
   bsa_status s = check_params(p, mode, param, &need);
   if (s != BSA_OK) return s;
@@ -248,6 +248,7 @@ bsa_status run_select(const bsa_plan_s* p, const float* qc, const float* kc, bsa
   bsa::SelectArgs a;
   std::memset(&a, 0, sizeof(a));
   a.qc = qc; a.kc = kc; a.idx = idx; a.cnt = cnt; a.scores = scores; a.kmax = kmax;
+  a.list_bits = list_bits;
   a.mode = (int)mode;
   a.est = est;
   if (map) a.map = *map;
@@ -375,9 +376,11 @@ float* text_part_of(const bsa_plan_s* p, int kmax, char* w) {
 
 // Pairs the query tiles of the selected heads (scratch and schedule carved
 // from `w`, pairing_bytes long); on return *sched / *lists point at them.
+// With bits_ready the lists' bit sets are already at the start of `w`
+// (written by the selection).
 bsa_status run_pairing(const bsa_plan_s* p, const int32_t* idx, const int32_t* cnt, int kmax,
                        char* w, int32_t** sched, int32_t** lists, cudaStream_t st,
-                       const bsa::HeadMap* map) {
+                       const bsa::HeadMap* map, bool bits_ready = false) {
   const size_t bh = (size_t)p->g.B * p->g.Hd, pph = pairs_per_head(p->g);
   const size_t nbw = (p->g.nb + 31) / 32;
   bsa::PairArgs pa;
@@ -393,6 +396,7 @@ bsa_status run_pairing(const bsa_plan_s* p, const int32_t* idx, const int32_t* c
   pa.kmax = kmax;
   pa.pairs_per_head = (int)pph;
   pa.text_pairs = text_pairs(p->g);
+  pa.bits_ready = bits_ready ? 1 : 0;
   if (map) pa.map = *map;
   cudaError_t e = bsa::launch_pairing(p->g, pa, st);
   if (e != cudaSuccess) return cuda_fail(e, "pairing kernels");
@@ -490,15 +494,17 @@ bsa_status run_forward_fused(const bsa_plan_s* p, const void* q, const void* k, 
   bsa_status s = run_centroids(p, q, k, qc, kc, st, k_sics, est != bsa::kEstMean, map);
   if (s != BSA_OK) return s;
   mark(timer);
+  // pairing only reorders the work; plans beyond its block limit run unpaired
+  const bool paired = pair_ws != nullptr && bsa::pairing_supported(p->g);
+  // the selection writes the lists' bit sets straight into the pairing scratch
+  uint32_t* list_bits = paired ? reinterpret_cast<uint32_t*>(pair_ws) : nullptr;
   if ((s = run_select(p, qc, kc, mode, param, kmax, idx, cnt, nullptr, st, uo, k_sics, bits, est,
-                      map)) != BSA_OK)
+                      map, list_bits)) != BSA_OK)
     return s;
   mark(timer);
   int32_t* sched = nullptr;
   int32_t* lists = nullptr;
-  // pairing only reorders the work; plans beyond its block limit run unpaired
-  if (pair_ws != nullptr && bsa::pairing_supported(p->g) &&
-      (s = run_pairing(p, idx, cnt, kmax, pair_ws, &sched, &lists, st, map)) != BSA_OK)
+  if (paired && (s = run_pairing(p, idx, cnt, kmax, pair_ws, &sched, &lists, st, map, true)) != BSA_OK)
     return s;
   mark(timer);
   s = run_attention_orig(p, q, k, v, idx, cnt, kmax, o, dev_status, st, map, sched, lists,

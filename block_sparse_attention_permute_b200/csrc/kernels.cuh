@@ -58,6 +58,7 @@ struct SelectArgs {
   int win_left, win_right;      // j in [i - left, i + right]; < 0 = unbounded; both < 0 = none
   long long sink_tokens;        // blocks holding any of the first sink_tokens tokens
   const uint32_t* intra_bits;   // [B, Hd, nbw] selected key blocks, or null
+  uint32_t* list_bits;          // [B * Hd, nb, nbw] out: each list's video blocks as a bit set, or null
   HeadMap map;
 };
 
@@ -126,6 +127,7 @@ struct PairArgs {
   int32_t* lists;         // [B * Hd, pairs_per_head, 2, kmax] out
   int kmax;
   int pairs_per_head, text_pairs;
+  int bits_ready;         // the bit sets were written by the selection (no bit-set pass)
   HeadMap map;            // pairs of (b, h) to pair up (n = 0: all)
 };
 

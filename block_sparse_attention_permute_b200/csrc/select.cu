@@ -403,7 +403,8 @@ __global__ void __launch_bounds__(kSelThreads, KMAX == 16 ? 3 : 2)
     const bool window = a.win_left >= 0 || a.win_right >= 0;
     const long long w_lo = a.win_left < 0 ? 0 : (long long)i - a.win_left;
     const long long w_hi = a.win_right < 0 ? nb : (long long)i + a.win_right;
-    const uint32_t* ibits = a.intra_bits ? a.intra_bits + bh * ((nb + 31) / 32) : nullptr;
+    const int nbw = (nb + 31) / 32;
+    const uint32_t* ibits = a.intra_bits ? a.intra_bits + bh * nbw : nullptr;
     for (int j0 = 0; j0 < nb; j0 += 32) {
       const int j = j0 + lane;
       const uint32_t key = j < nb ? order_key(row[j]) : 0u;
@@ -418,6 +419,7 @@ __global__ void __launch_bounds__(kSelThreads, KMAX == 16 ? 3 : 2)
       }
       const uint32_t sel_bal = __ballot_sync(0xffffffffu, take);
       if (take) out[written + __popc(sel_bal & lt_mask)] = j;
+      if (a.list_bits != nullptr && lane == 0) a.list_bits[(bh * nb + i) * nbw + (j0 >> 5)] = sel_bal;
       written += __popc(sel_bal);
       eq_seen += __popc(eq_bal);
     }

@@ -138,3 +138,41 @@ def test_pair_schedule_full_hunyuan(dev):
     frac = shared / video
     print(f"hunyuan: matched pairs share {frac:.3f} of their video blocks")
     assert frac >= 0.5
+
+
+@pytest.mark.parametrize("name", ["hy_ragged_text", "wan_d64_b2", "wan_topp", "window_lt_nb"])
+def test_forward_pairing_equals_pair_tiles(name, dev):
+    """bsa_forward hands the pairing the bit sets the selection writes beside
+    its lists (no separate bit-set pass): the bit sets, the schedule and the
+    reordered lists in the forward's workspace equal those bsa_pair_tiles
+    derives from the same lists, bit for bit."""
+    w = CASES[name]
+    q, k, v = synthetic.make_qkv(w)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    plan = bsa.plan_for(w, dev)
+    kmax = plan.kmax_for(w.mode, w.params)
+    ws = torch.zeros(plan.workspace_size(kmax)[1], dtype=torch.uint8, device=dev)
+    _, idx, cnt = plan.forward(qd, kd, vd, w.mode, w.params, kmax=kmax, workspace=ws,
+                               return_lists=True)
+    ref = plan.pair_tiles(idx, cnt)
+    plan.check_status()
+    info = plan.info
+    bh, nb = info.batch * info.heads, info.nb
+    # the forward's workspace: Q and K centroids, its own lists and counts, then
+    # the pairing workspace
+    off = 2 * _r256(bh * nb * info.head_dim * 4) + _r256(bh * nb * kmax * 4) + _r256(bh * nb * 4)
+    fwd = ws[off:]
+    nbits = bh * nb * ((nb + 31) // 32) * 4
+    assert torch.equal(fwd[:nbits].cpu(), ref[:nbits].cpu())
+    sched_f, lists_f, tp = read_schedule(plan, fwd, kmax)
+    sched_r, lists_r, _ = read_schedule(plan, ref, kmax)
+    assert np.array_equal(sched_f, sched_r)
+    cnt_np = cnt.cpu().numpy().reshape(bh, nb)
+    for b in range(bh):
+        for e in range(tp, sched_r.shape[1]):
+            for x in range(2):
+                t = int(sched_r[b, e, x])
+                if t >= 0:
+                    n = cnt_np[b, t]
+                    assert np.array_equal(lists_f[b, e, x, :n], lists_r[b, e, x, :n]), (b, e, x)
+    check_schedule(plan, idx, cnt, fwd)
