@@ -474,8 +474,8 @@ def time_workload(bsa, name, dev, barrier, args, cache, peak_burst, peak_sust):
         else:
             calls += [lambda: L.bsa_attention_orig(plan._h, P(qd), P(kd), P(vd), P(idx), P(cnt), kmax,
                                                    P(out), None, S())]
-        # per bsa_forward step: centroids, select, 2 pairing kernels, attention, text merge
-        launches = 3 + (2 if paired else 0) + (1 if paired and plan.info.nb_text > 0 else 0)
+        # per bsa_forward step: centroids, select, 3 pairing kernels, attention, text merge
+        launches = 3 + (3 if paired else 0) + (1 if paired and plan.info.nb_text > 0 else 0)
     else:
         qb, kb, vb, ob = (torch.empty(plan.blk_shape, dtype=plan.dtype, device=dev) for _ in range(4))
         names = ["permute", "select", "attention", "unpermute"]
@@ -836,11 +836,11 @@ def run_ours(args, rank, world, local):
                                   frac=round(scheme["achieved_gbs"] / hbm_gbs, 4),
                                   peak_gbs=hbm_gbs, bound="hbm"),
         # per bsa_forward step, tensor-core plans: centroids, select (which also
-        # writes the lists' bit sets), 2 pairing kernels (candidates; matching
-        # with the reordered lists; none beyond 1536 video blocks), attention,
-        # and with text tokens the merge of the text chunks; other plans:
-        # permute, select, attention, unpermute
-        "gpu_launches": ((3 + (2 if plan.info.nb <= 1536 else 0)
+        # writes the lists' bit sets), 3 pairing kernels (candidates, matching,
+        # reordered lists; none beyond 1536 video blocks), attention, and with
+        # text tokens the merge of the text chunks; other plans: permute,
+        # select, attention, unpermute
+        "gpu_launches": ((3 + (3 if plan.info.nb <= 1536 else 0)
                           + (1 if plan.info.nb <= 1536 and plan.info.nb_text > 0 else 0))
                          if plan.info.attn_path == 1 else 4) * args.steps,
         "clocks": clocks,

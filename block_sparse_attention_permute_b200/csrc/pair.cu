@@ -187,7 +187,7 @@ __device__ __forceinline__ int write_bits(const uint32_t* wordsA, const uint32_t
 }
 
 // Matching of one (b, h): one CTA of 1024 threads, in shared memory; writes
-// every schedule entry and the reordered lists of its two tiles.
+// the tiles of every schedule entry.
 __global__ void __launch_bounds__(1024) pair_match_kernel(Geo g, PairArgs a) {
   extern __shared__ int sm_pair[];
   const int nb = g.nb;
@@ -261,40 +261,48 @@ __global__ void __launch_bounds__(1024) pair_match_kernel(Geo g, PairArgs a) {
     sched[t * 4 + 2] = i1 >= 0 ? nb + g.nb_text : 0;
     sched[t * 4 + 3] = 0;
   }
-  // Video pairs, one warp per pair: the reordered lists — the shared video
-  // blocks, the text blocks, then each tile's own blocks, all ascending —
-  // and the entry (tiles, shared count c).
-  const int nbw = (nb + 31) / 32;
-  const uint32_t* bits = a.bits + (long long)bh * nb * nbw;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int p = warp; p < a.pairs_per_head - a.text_pairs; p += blockDim.x >> 5) {
+  // video pairs: the tiles here, the shared count with the lists (next kernel)
+  for (int p = threadIdx.x; p < a.pairs_per_head - a.text_pairs; p += blockDim.x) {
     const int e = a.text_pairs + p;
-    const int i = p < np ? pair_i[p] : -1, j = p < np ? pair_j[p] : -1;
-    int c = 0;
-    if (i >= 0) {
-      const uint32_t* bi = bits + (long long)i * nbw;
-      int32_t* li = a.lists + ((long long)bh * a.pairs_per_head + e) * 2 * a.kmax;
-      int32_t* lj = li + a.kmax;
-      if (j >= 0) {
-        const uint32_t* bj = bits + (long long)j * nbw;
-        const int ns = write_bits(bi, bj, false, true, nbw, li, 0, lane);
-        write_bits(bi, bj, false, true, nbw, lj, 0, lane);
-        for (int t = lane; t < g.nb_text; t += 32) { li[ns + t] = nb + t; lj[ns + t] = nb + t; }
-        c = ns + g.nb_text;
-        write_bits(bi, bj, true, false, nbw, li, c, lane);
-        write_bits(bj, bi, true, false, nbw, lj, c, lane);
-      } else {
-        const int ns = write_bits(bi, bi, false, false, nbw, li, 0, lane);
-        for (int t = lane; t < g.nb_text; t += 32) li[ns + t] = nb + t;
-      }
-    }
-    if (lane == 0) {
-      sched[e * 4 + 0] = i;
-      sched[e * 4 + 1] = j;
-      sched[e * 4 + 2] = c;
-      sched[e * 4 + 3] = 0;
-    }
+    sched[e * 4 + 0] = p < np ? pair_i[p] : -1;
+    sched[e * 4 + 1] = p < np ? pair_j[p] : -1;
+    sched[e * 4 + 2] = 0;
+    sched[e * 4 + 3] = 0;
   }
+}
+
+// Reordered lists of every video pair (one warp per pair): the shared video
+// blocks, the text blocks, then each tile's own blocks, all ascending; the
+// shared count c goes into the schedule entry.
+__global__ void __launch_bounds__(256) pair_lists_kernel(Geo g, PairArgs a) {
+  const int vp = a.pairs_per_head - a.text_pairs;
+  const int p = blockIdx.y * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (p >= vp) return;
+  const int bh = map_bh(a.map, blockIdx.x);
+  const int nb = g.nb, nbw = (nb + 31) / 32;
+  const int e = a.text_pairs + p;
+  int32_t* ent = a.sched + ((long long)bh * a.pairs_per_head + e) * 4;
+  const int i = ent[0], j = ent[1];
+  if (i < 0) return;
+  const uint32_t* bits = a.bits + (long long)bh * nb * nbw;
+  const uint32_t* bi = bits + (long long)i * nbw;
+  int32_t* lists = a.lists + ((long long)bh * a.pairs_per_head + e) * 2 * a.kmax;
+  int32_t* li = lists;
+  int32_t* lj = lists + a.kmax;
+  int c = 0;
+  if (j >= 0) {
+    const uint32_t* bj = bits + (long long)j * nbw;
+    const int ns = write_bits(bi, bj, false, true, nbw, li, 0, lane);
+    write_bits(bi, bj, false, true, nbw, lj, 0, lane);
+    for (int t = lane; t < g.nb_text; t += 32) { li[ns + t] = nb + t; lj[ns + t] = nb + t; }
+    c = ns + g.nb_text;
+    write_bits(bi, bj, true, false, nbw, li, c, lane);
+    write_bits(bj, bi, true, false, nbw, lj, c, lane);
+  } else {
+    const int ns = write_bits(bi, bi, false, false, nbw, li, 0, lane);
+    for (int t = lane; t < g.nb_text; t += 32) li[ns + t] = nb + t;
+  }
+  if (lane == 0) ent[2] = c;
 }
 
 cudaError_t launch_pairing(const Geo& g, const PairArgs& a, cudaStream_t st) {
@@ -302,7 +310,7 @@ cudaError_t launch_pairing(const Geo& g, const PairArgs& a, cudaStream_t st) {
   if (n_bh == 0 || g.nb == 0) return cudaSuccess;
   if (g.nb > 32 * kMaxWords) return cudaErrorInvalidValue;
   cudaError_t e;
-  if (!a.bits_ready) {
+  if (!a.bits_ready) {   // else the selection wrote the bit sets with the lists
     pair_bits_kernel<<<dim3(n_bh, (g.nb + 7) / 8), 256, 0, st>>>(g, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -318,6 +326,9 @@ cudaError_t launch_pairing(const Geo& g, const PairArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
   }
   pair_match_kernel<<<n_bh, 1024, smem, st>>>(g, a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int vp = a.pairs_per_head - a.text_pairs;
+  pair_lists_kernel<<<dim3(n_bh, (vp + 7) / 8), 256, 0, st>>>(g, a);
   return cudaGetLastError();
 }
 
