@@ -138,7 +138,9 @@ def box_summaries(g: Geometry, x):
 
 
 def scores_box(g: Geometry, qbox, kbox, variant: int):
-    """Row softmax of the DSA (variant 1) or DSA2 (variant 2) estimate / sqrt(D)."""
+    """Row softmax of the DSA (variant 1) or DSA2 (variant 2) estimate / sqrt(D).
+    Parity unpinned: the estimator is a reading of SPADE §3.1 / Fig. 4 (the
+    equations are not in the text), pinned only to a corner brute force."""
     qbox = np.ascontiguousarray(qbox, dtype=np.float64)
     kbox = np.ascontiguousarray(kbox, dtype=np.float64)
     out = np.empty((g.B, g.Hd, g.nb, g.nb), dtype=np.float64)

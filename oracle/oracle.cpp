@@ -44,7 +44,10 @@
 //   R20 intra scores: one per key block, broadcast to every query block of
 //       the head; selected by the Top-K / Top-P rule on the scores.
 //   R21 DSA / DSA2 inter-estimators: the largest q . k over the summaries'
-//       boxes (DSA: query fixed at the box centre).
+//       boxes (DSA: query fixed at the box centre).  Parity unpinned: the
+//       pages give the summaries but not the estimator equations, so
+//       orc_scores_box is checked against this reading (a brute force over
+//       the box corners), not against a value or formula of the pages.
 //
 // Geometry array g[10] = {B, T, H, W, bf, br, bc, Hd, D, n_text}.
 
