@@ -897,6 +897,10 @@ bsa_status bsa_forward_timed(bsa_plan_t p, const void* q, const void* k, const v
   bsa_status s = forward_impl(p, q, k, v, mode, param, nullptr, kmax, o, idx_out, cnt_out, ws,
                               ws_bytes, dev_status, stream, bsa::kEstMean, &t);
   if (s == BSA_OK && t.err != cudaSuccess) s = cuda_fail(t.err, "cudaEventRecord");
+  if (s == BSA_OK && t.n < 2) {   // nothing was launched: every phase took 0 ms
+    destroy();
+    return s;
+  }
   if (s == BSA_OK && (e = cudaEventSynchronize(t.ev[t.n - 1])) != cudaSuccess) s = cuda_fail(e, "cudaEventSynchronize");
   if (s == BSA_OK) {
     float ms[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
